@@ -1,0 +1,187 @@
+/*
+ * tq.h -- C ABI of libtq, a B200 (sm_100a) implementation of the TurboQuant
+ * KV-cache vector compression hot path.
+ *
+ * What the method computes (web pages on the turboquant-pytorch / turboquant-py
+ * implementations of Google's TurboQuant):
+ *   - stage 1 ("TurboQuantMSE"): normalise a vector, rotate it by a fixed random
+ *     orthogonal matrix R so every coordinate follows N(0, 1/d), and Lloyd-Max
+ *     quantize each coordinate with b bits
+ *       ["turboquant-pytorch" (atskills.one), "What It Does" and
+ *        "Algorithm Details: Why Random Rotation?";
+ *        "turboquant-pytorch" (nav.superapi.store), 主要能力, 核心 API, 算法细节];
+ *   - stage 2 ("TurboQuantProd", keys only): a 1-bit QJL sign sketch of the residual
+ *     through a Gaussian matrix S with proj_dim = head_dim/2 rows, which makes inner
+ *     product estimates unbiased [same pages, "Why QJL for Keys but Not Values?",
+ *     算法细节 "proj_dim 选择"];
+ *   - attention straight from the compressed keys ("asymmetric_attention_scores"),
+ *     softmax, weighted sum over the MSE-dequantized values
+ *       [nav.superapi.store page, 常见使用模式 "压缩整个模型的 KV 缓存"].
+ *
+ * Conventions (all functions):
+ *   - Every call returns a tq_status.  Argument errors are detected on the host and
+ *     returned before anything is launched; nothing is written in that case.
+ *   - The caller allocates and owns every buffer.  The library never allocates,
+ *     frees or keeps device memory and holds no global mutable state.
+ *   - Device work is enqueued asynchronously on the caller's stream; results are
+ *     ready when that stream is synchronised.  Outputs are bit-identical run to run.
+ *   - Device pointers must be 16-byte aligned (TQ_ERR_INVALID_ARG otherwise).
+ *   - dev_status (optional, may be NULL) is a device int32 that kernels set to a
+ *     nonzero tq_status if they detect an error on the device; it is never cleared
+ *     by the library.
+ *
+ * Packed layout (a contract of this library; the pages do not fix one):
+ *   codes  : per vector, dim/32 groups of beta little-endian uint32 words; word
+ *            g*beta + p holds bit p of the code of coordinate 32g+l at bit l
+ *            (beta = bits-1 for keys, bits for values);
+ *   signs  : per key, proj_dim/32 words; word g bit l = [p_{32g+l} >= 0];
+ *   norms  : IEEE binary16 (round to nearest even) of the fp32 value.
+ *   Keys take (bits-1)*dim/8 + proj_dim/8 + 4 bytes, values bits*dim/8 + 2 bytes.
+ *   Records of a cache are ordered [B, Hkv, T] (row-major).
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *tq_stream_t; /* binary-compatible with cudaStream_t */
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or value      */
+    TQ_ERR_UNSUPPORTED = 2, /* valid arguments outside what the kernels implement */
+    TQ_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed               */
+    TQ_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (dev_status)    */
+} tq_status;
+
+typedef enum tq_dtype { TQ_F16 = 0, TQ_F32 = 1 } tq_dtype;
+
+/* Human-readable name of a status code.  Never returns NULL. */
+const char *tq_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int tq_version(void);
+
+/*
+ * Lloyd-Max codebook for one coordinate of a randomly rotated unit vector, whose law
+ * is taken as N(0, 1/dim) (nav.superapi.store page, 核心 API
+ * "build_lloyd_max_codebook(dim=128, bits=3) returns (boundaries, centroids)";
+ * atskills.one page, "Why Random Rotation?").  HOST function, no device work.
+ *   dim        : vector dimension (>= 1)
+ *   bits       : 1..4
+ *   boundaries : host array of 2^bits - 1 floats, ascending; the middle one is 0
+ *   centroids  : host array of 2^bits floats, ascending, antisymmetric
+ * A coordinate y gets code #{k : boundaries[k] < y} (ties go to the lower cell).
+ */
+tq_status tq_codebook(int dim, int bits, float *boundaries, float *centroids);
+
+/*
+ * Quantizer parameters.  R and S are caller-generated (the pages use a fixed random
+ * orthogonal R and an i.i.d. N(0,1) matrix S; the library takes them as inputs).
+ *   dim      : head dimension d; a multiple of 32, 32..1024
+ *   bits     : nominal bits per coordinate b, 1..4.  Values use b MSE bits; keys use
+ *              b-1 MSE bits plus one QJL sign per projection (so keys need b >= 2)
+ *   proj_dim : QJL projection count m; a multiple of 32, 32..1024 (0 = values only)
+ *   R        : device fp32 [dim, dim], row-major, orthogonal; rotation y = R u
+ *   S        : device fp32 [proj_dim, dim], row-major (NULL when proj_dim == 0)
+ *   workspace: device buffer of at least tq_workspace_bytes(dim, bits, proj_dim)
+ *              bytes, filled by tq_prepare; read by every other call
+ */
+typedef struct tq_params {
+    int dim;
+    int bits;
+    int proj_dim;
+    const float *R;
+    const float *S;
+    void *workspace;
+    size_t workspace_bytes;
+} tq_params;
+
+/* Bytes of workspace tq_prepare needs for these sizes (0 if the sizes are invalid). */
+size_t tq_workspace_bytes(int dim, int bits, int proj_dim);
+
+/*
+ * Derive everything the kernels need from (R, S, codebooks) into p->workspace:
+ * the fp32 codebooks for bits-1 and bits, S' = S R^T (the QJL projection expressed on
+ * rotated coordinates) and the split-precision operand copies of R and S'.  Call it
+ * once per (R, S), and again whenever they change.  Enqueued on `stream`.
+ */
+tq_status tq_prepare(const tq_params *p, int32_t *dev_status, tq_stream_t stream);
+
+/*
+ * Compress n key vectors (TurboQuantProd.compress / TurboQuantCompressorV2;
+ * nav.superapi.store page, 核心 API; atskills.one page, "What It Does" stages 1+2):
+ *   n_k = ||x||, u = x / n_k, y = R u, idx_j = code of y_j with the (dim, bits-1)
+ *   codebook, e = y - c[idx] (so the residual r = R^T e), rho = ||e||,
+ *   sign_i = [ (S r)_i >= 0 ].
+ *   x      : device [n, dim], fp16 or fp32 (dtype), row-major
+ *   codes  : device uint32 [n, (bits-1)*dim/32]
+ *   signs  : device uint32 [n, proj_dim/32]
+ *   norm   : device fp16 bits [n]  (||x||)
+ *   rnorm  : device fp16 bits [n]  (||r|| of the unit vector's residual)
+ * n may be 0 (no work).  A zero vector gets norm 0 and the codes of y = 0.
+ */
+tq_status tq_compress_keys(const tq_params *p, const void *x, tq_dtype dtype, int64_t n,
+                           uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
+                           int32_t *dev_status, tq_stream_t stream);
+
+/*
+ * Compress n value vectors (TurboQuantMSE.quantize / TurboQuantCompressorMSE: stage 1
+ * only; atskills.one page, "Why QJL for Keys but Not Values?").
+ *   codes : device uint32 [n, bits*dim/32];  norm : device fp16 bits [n]
+ */
+tq_status tq_compress_values(const tq_params *p, const void *x, tq_dtype dtype, int64_t n,
+                             uint32_t *codes, uint16_t *norm, int32_t *dev_status,
+                             tq_stream_t stream);
+
+/*
+ * Asymmetric inner-product estimates straight from packed keys
+ * (TurboQuantProd.inner_product / asymmetric_attention_scores; nav.superapi.store page,
+ * 核心 API and 常见使用模式):
+ *   s = ||k|| * ( <R q, c[idx]> + rho * sqrt(pi/2)/proj_dim * <S q, 2*sign - 1> )
+ * (the raw estimate of <q, k>; no 1/sqrt(d) scaling).
+ *   q      : device fp32 [B, Hq, Nq, dim];  query head h reads KV head h / (Hq/Hkv)
+ *   keys   : the four arrays of tq_compress_keys for [B, Hkv, T] records
+ *   scores : device fp32 [B, Hq, Nq, T], or NULL when only top-k is wanted
+ *   topk   : 0, or 1..64: also return the topk largest scores of every (b, h, query)
+ *            row, descending, ties to the smaller token index
+ *   topk_idx / topk_val : device int32 / fp32 [B, Hq, Nq, topk] (when topk > 0)
+ *   scratch: device buffer of tq_scores_scratch_bytes(...) bytes (may be NULL if 0)
+ */
+size_t tq_scores_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T,
+                               int topk);
+tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx,
+                    float *topk_val, void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                    tq_stream_t stream);
+
+/*
+ * Attention over a compressed cache, fused: scores from the packed keys, softmax of
+ * scale*scores over all T tokens (no mask), weighted sum of the dequantized values
+ * (nav.superapi.store page, 常见使用模式: "softmax 后对解压的值做加权求和"):
+ *   out = sum_t softmax_t(scale * s_t) * ||v_t|| * R^T c[vidx_t]
+ *   q      : device fp32 [B, Hq, Nq, dim]
+ *   keys   : as tq_scores;  vcodes / vnorm: the arrays of tq_compress_values
+ *   scale  : softmax temperature; <= 0 selects 1/sqrt(dim)
+ *   out    : device fp32 [B, Hq, Nq, dim]
+ *   scratch: device buffer of tq_attend_scratch_bytes(...) bytes (split-context partials)
+ * T must be >= 1.
+ */
+size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T);
+tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm,
+                    float scale, float *out, void *scratch, size_t scratch_bytes,
+                    int32_t *dev_status, tq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */
