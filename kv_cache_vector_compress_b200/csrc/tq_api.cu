@@ -1,0 +1,236 @@
+// tq_api.cu -- the extern "C" entry points of libtq: argument checks, then launches.
+#include <cmath>
+#include <cstring>
+
+#include "tq_internal.cuh"
+
+using namespace tq;
+
+namespace {
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool dim_supported(int d) {
+    return d == 32 || d == 64 || d == 128 || d == 256 || d == 512 || d == 1024;
+}
+
+// Common checks on a parameter set; `need_keys` requires the QJL part.
+tq_status check_params(const tq_params *p, bool need_keys) {
+    if (!p) return TQ_ERR_INVALID_ARG;
+    if (p->dim < 32 || p->dim > kMaxDim || p->dim % 32) return TQ_ERR_INVALID_ARG;
+    if (p->bits < 1 || p->bits > 4) return TQ_ERR_INVALID_ARG;
+    if (p->proj_dim < 0 || p->proj_dim > kMaxProj || p->proj_dim % 32) return TQ_ERR_INVALID_ARG;
+    if (need_keys && (p->bits < 2 || p->proj_dim < 32)) return TQ_ERR_INVALID_ARG;
+    if (!p->workspace || !aligned16(p->workspace)) return TQ_ERR_INVALID_ARG;
+    if (p->workspace_bytes < ws_layout(p->dim, p->proj_dim).total) return TQ_ERR_INVALID_ARG;
+    if (!dim_supported(p->dim)) return TQ_ERR_UNSUPPORTED;
+    return TQ_OK;
+}
+
+tq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+tq_status check_problem(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T, const float *q,
+                        const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                        const uint16_t *krnorm) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || T < 1 || Hq % Hkv) return TQ_ERR_INVALID_ARG;
+    if (T > (int64_t)INT32_MAX) return TQ_ERR_UNSUPPORTED;
+    // every index used by the kernels must fit in int64 comfortably
+    const double recs = (double)B * Hkv * (double)T, rows = (double)B * Hq * Nq;
+    if (recs * p->dim > 9e18 || rows * (double)T > 9e18) return TQ_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, kcodes, ksigns, knorm, krnorm};
+    for (const void *x : ptrs)
+        if (!x || !aligned16(x)) return TQ_ERR_INVALID_ARG;
+    return TQ_OK;
+}
+
+ScoreProblem make_problem(int B, int Hq, int Hkv, int Nq, int64_t T, const float *q, const uint32_t *kcodes,
+                          const uint32_t *ksigns, const uint16_t *knorm, const uint16_t *krnorm,
+                          const uint32_t *vcodes, const uint16_t *vnorm) {
+    ScoreProblem sp;
+    sp.B = B;
+    sp.Hq = Hq;
+    sp.Hkv = Hkv;
+    sp.Nq = Nq;
+    sp.T = T;
+    sp.q = q;
+    sp.kcodes = kcodes;
+    sp.ksigns = ksigns;
+    sp.knorm = knorm;
+    sp.krnorm = krnorm;
+    sp.vcodes = vcodes;
+    sp.vnorm = vnorm;
+    return sp;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tq_status_string(int status) {
+    switch (status) {
+        case TQ_OK: return "TQ_OK";
+        case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+        case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+        case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+        case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT";
+        default: return "TQ_ERR_UNKNOWN";
+    }
+}
+
+int tq_version(void) { return 100; }
+
+tq_status tq_codebook(int dim, int bits, float *boundaries, float *centroids) {
+    if (dim < 1 || bits < 1 || bits > 4 || !boundaries || !centroids) return TQ_ERR_INVALID_ARG;
+    double b[kMaxLevels], c[kMaxLevels];
+    if (lloyd_max_gaussian(dim, bits, b, c) < 0) return TQ_ERR_INVALID_ARG;
+    const int K = 1 << bits;
+    for (int k = 0; k < K - 1; ++k) boundaries[k] = (float)b[k];
+    for (int k = 0; k < K; ++k) centroids[k] = (float)c[k];
+    return TQ_OK;
+}
+
+size_t tq_workspace_bytes(int dim, int bits, int proj_dim) {
+    if (dim < 32 || dim > kMaxDim || dim % 32 || bits < 1 || bits > 4) return 0;
+    if (proj_dim < 0 || proj_dim > kMaxProj || proj_dim % 32) return 0;
+    return ws_layout(dim, proj_dim).total;
+}
+
+tq_status tq_prepare(const tq_params *p, int32_t *dev_status, tq_stream_t stream) {
+    (void)dev_status;
+    tq_status st = check_params(p, false);
+    if (st != TQ_OK) return st;
+    if (!p->R || !aligned16(p->R)) return TQ_ERR_INVALID_ARG;
+    if (p->proj_dim > 0 && (!p->S || !aligned16(p->S))) return TQ_ERR_INVALID_ARG;
+    Codebooks cb;
+    memset(&cb, 0, sizeof(cb));
+    double b[kMaxLevels], c[kMaxLevels];
+    const int K = 1 << p->bits;
+    if (lloyd_max_gaussian(p->dim, p->bits, b, c) < 0) return TQ_ERR_INVALID_ARG;
+    for (int k = 0; k < K; ++k) {
+        cb.vc[k] = (float)c[k];
+        if (k < K - 1) cb.vb[k] = (float)b[k];
+    }
+    // unused boundary slots never count: +inf is never below a finite value
+    for (int k = K - 1; k < kMaxLevels; ++k) cb.vb[k] = INFINITY;
+    if (p->bits >= 2) {
+        const int Kk = K / 2;
+        if (lloyd_max_gaussian(p->dim, p->bits - 1, b, c) < 0) return TQ_ERR_INVALID_ARG;
+        for (int k = 0; k < Kk; ++k) {
+            cb.kc[k] = (float)c[k];
+            if (k < Kk - 1) cb.kb[k] = (float)b[k];
+        }
+        for (int k = Kk - 1; k < kMaxLevels; ++k) cb.kb[k] = INFINITY;
+    } else {
+        for (int k = 0; k < kMaxLevels; ++k) cb.kb[k] = INFINITY;
+    }
+    return from_cuda(launch_prepare(p, cb, (cudaStream_t)stream));
+}
+
+tq_status tq_compress_keys(const tq_params *p, const void *x, tq_dtype dtype, int64_t n, uint32_t *codes,
+                           uint32_t *signs, uint16_t *norm, uint16_t *rnorm, int32_t *dev_status,
+                           tq_stream_t stream) {
+    tq_status st = check_params(p, true);
+    if (st != TQ_OK) return st;
+    if (dtype != TQ_F16 && dtype != TQ_F32) return TQ_ERR_INVALID_ARG;
+    if (n < 0) return TQ_ERR_INVALID_ARG;
+    if (n == 0) return TQ_OK;
+    const void *ptrs[] = {x, codes, signs, norm, rnorm};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    return from_cuda(launch_compress(P, true, x, dtype == TQ_F16, n, codes, signs, norm, rnorm, dev_status,
+                                     (cudaStream_t)stream));
+}
+
+tq_status tq_compress_values(const tq_params *p, const void *x, tq_dtype dtype, int64_t n, uint32_t *codes,
+                             uint16_t *norm, int32_t *dev_status, tq_stream_t stream) {
+    tq_status st = check_params(p, false);
+    if (st != TQ_OK) return st;
+    if (dtype != TQ_F16 && dtype != TQ_F32) return TQ_ERR_INVALID_ARG;
+    if (n < 0) return TQ_ERR_INVALID_ARG;
+    if (n == 0) return TQ_OK;
+    const void *ptrs[] = {x, codes, norm};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    return from_cuda(launch_compress(P, false, x, dtype == TQ_F16, n, codes, nullptr, norm, nullptr,
+                                     dev_status, (cudaStream_t)stream));
+}
+
+size_t tq_scores_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T, int topk) {
+    if (check_params(p, true) != TQ_OK) return 0;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || T < 1 || Hq % Hkv) return 0;
+    Prepared P = prepared_view(p);
+    ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                   nullptr);
+    size_t bytes = qprep_bytes(P, sp);
+    if (topk > 0) bytes += topk_scratch_bytes(P, sp, topk);
+    return bytes;
+}
+
+tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx, float *topk_val,
+                    void *scratch, size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
+    (void)dev_status;
+    tq_status st = check_params(p, true);
+    if (st != TQ_OK) return st;
+    st = check_problem(p, B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm);
+    if (st != TQ_OK) return st;
+    if (topk < 0 || topk > kMaxTopk || topk > T) return TQ_ERR_INVALID_ARG;
+    if (topk == 0 && !scores) return TQ_ERR_INVALID_ARG;
+    if (scores && !aligned16(scores)) return TQ_ERR_INVALID_ARG;
+    if (topk > 0 && (!topk_idx || !topk_val || !aligned16(topk_idx) || !aligned16(topk_val)))
+        return TQ_ERR_INVALID_ARG;
+    if (!scratch || !aligned16(scratch)) return TQ_ERR_INVALID_ARG;
+    if (scratch_bytes < tq_scores_scratch_bytes(p, B, Hq, Hkv, Nq, T, topk)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm, nullptr, nullptr);
+    cudaStream_t s = (cudaStream_t)stream;
+    float *qprep = (float *)scratch;
+    float *sbuf = scores;
+    if (!sbuf) sbuf = (float *)((char *)scratch + qprep_bytes(P, sp));
+    cudaError_t e = launch_qprep(P, sp, qprep, s);
+    if (e == cudaSuccess) e = launch_scores(P, sp, qprep, sbuf, s);
+    if (e == cudaSuccess && topk > 0) e = launch_topk(sp, sbuf, topk, topk_idx, topk_val, s);
+    return from_cuda(e);
+}
+
+size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T) {
+    if (check_params(p, true) != TQ_OK) return 0;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || T < 1 || Hq % Hkv) return 0;
+    Prepared P = prepared_view(p);
+    ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                   nullptr);
+    return qprep_bytes(P, sp) + attend_partials_bytes(P, sp, nullptr);
+}
+
+tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm, float scale,
+                    float *out, void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                    tq_stream_t stream) {
+    (void)dev_status;
+    tq_status st = check_params(p, true);
+    if (st != TQ_OK) return st;
+    st = check_problem(p, B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm);
+    if (st != TQ_OK) return st;
+    if (!vcodes || !vnorm || !out || !aligned16(vcodes) || !aligned16(vnorm) || !aligned16(out))
+        return TQ_ERR_INVALID_ARG;
+    if (!(scale == scale)) return TQ_ERR_INVALID_ARG;  // NaN
+    if (!scratch || !aligned16(scratch)) return TQ_ERR_INVALID_ARG;
+    if (scratch_bytes < tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, T)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm, vcodes, vnorm);
+    if (scale <= 0.f) scale = 1.0f / sqrtf((float)p->dim);
+    cudaStream_t s = (cudaStream_t)stream;
+    float *qprep = (float *)scratch;
+    int splits = 1;
+    attend_partials_bytes(P, sp, &splits);
+    float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
+    cudaError_t e = launch_qprep(P, sp, qprep, s);
+    if (e == cudaSuccess) e = launch_attend(P, sp, qprep, scale, partials, splits, out, s);
+    return from_cuda(e);
+}
+
+}  // extern "C"

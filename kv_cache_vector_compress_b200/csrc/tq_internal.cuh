@@ -1,0 +1,118 @@
+// tq_internal.cuh -- definitions shared by the host code and the kernels of libtq.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kMaxDim = 1024;
+constexpr int kMaxProj = 1024;
+constexpr int kMaxLevels = 16;  // 4 bits
+constexpr int kMaxTopk = 64;
+constexpr uint32_t kWsMagic = 0x54513031u;  // "TQ01"
+
+// Codebooks of one prepared parameter set, as the kernels read them.
+struct Codebooks {
+    float kb[kMaxLevels];  // key boundaries (K-1 used)
+    float kc[kMaxLevels];  // key centroids
+    float vb[kMaxLevels];  // value boundaries
+    float vc[kMaxLevels];  // value centroids
+};
+
+// Byte offsets of the prepared arrays inside the caller's workspace.
+struct WsLayout {
+    size_t header;     // WsHeader
+    size_t codebooks;  // Codebooks
+    size_t R;          // fp32 [d, d]      copy of R
+    size_t RT;         // fp32 [d, d]      R transposed
+    size_t ST;         // fp32 [d, m]      S transposed
+    size_t SpT;        // fp32 [d, m]      (S R^T) transposed
+    size_t total;
+};
+
+struct WsHeader {
+    uint32_t magic;
+    int32_t dim, bits, proj_dim;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int d, int m) {
+    WsLayout L;
+    size_t o = 0;
+    L.header = o;
+    o = align_up(o + sizeof(WsHeader), 256);
+    L.codebooks = o;
+    o = align_up(o + sizeof(Codebooks), 256);
+    L.R = o;
+    o = align_up(o + sizeof(float) * (size_t)d * d, 256);
+    L.RT = o;
+    o = align_up(o + sizeof(float) * (size_t)d * d, 256);
+    L.ST = o;
+    o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 256);
+    L.SpT = o;
+    o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 256);
+    L.total = o;
+    return L;
+}
+
+// Device views of a prepared parameter set.
+struct Prepared {
+    int d, m, kbeta, vbeta;
+    const Codebooks *cb;
+    const float *R, *RT, *ST, *SpT;
+};
+
+inline Prepared prepared_view(const tq_params *p) {
+    WsLayout L = ws_layout(p->dim, p->proj_dim);
+    const char *w = (const char *)p->workspace;
+    Prepared v;
+    v.d = p->dim;
+    v.m = p->proj_dim;
+    v.kbeta = p->bits - 1;
+    v.vbeta = p->bits;
+    v.cb = (const Codebooks *)(w + L.codebooks);
+    v.R = (const float *)(w + L.R);
+    v.RT = (const float *)(w + L.RT);
+    v.ST = (const float *)(w + L.ST);
+    v.SpT = (const float *)(w + L.SpT);
+    return v;
+}
+
+// Host-side Lloyd-Max (tq_codebook.cpp).
+int lloyd_max_gaussian(int dim, int bits, double *bounds, double *cents);
+
+// Kernel launchers (tq_*.cu).  All return a cudaError_t from cudaGetLastError.
+cudaError_t launch_prepare(const tq_params *p, const Codebooks &cb, cudaStream_t s);
+cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
+                            uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
+                            int32_t *dev_status, cudaStream_t s);
+
+struct ScoreProblem {
+    int B, Hq, Hkv, Nq;
+    int64_t T;
+    const float *q;
+    const uint32_t *kcodes, *ksigns;
+    const uint16_t *knorm, *krnorm;
+    const uint32_t *vcodes;
+    const uint16_t *vnorm;
+};
+
+size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp);
+size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int *splits_out);
+size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
+
+cudaError_t launch_qprep(const Prepared &P, const ScoreProblem &sp, float *qprep, cudaStream_t s);
+cudaError_t launch_scores(const Prepared &P, const ScoreProblem &sp, const float *qprep,
+                          float *scores, cudaStream_t s);
+cudaError_t launch_topk(const ScoreProblem &sp, const float *scores, int topk, int32_t *idx,
+                        float *val, cudaStream_t s);
+cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float *qprep,
+                          float scale, float *partials, int splits, float *out, cudaStream_t s);
+
+}  // namespace tq

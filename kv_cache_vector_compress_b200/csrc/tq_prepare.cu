@@ -1,0 +1,57 @@
+// tq_prepare.cu -- derive the kernels' operand copies of R and S into the workspace.
+#include "tq_internal.cuh"
+
+namespace tq {
+
+namespace {
+
+__global__ void prepare_kernel(const float *__restrict__ R, const float *__restrict__ S, int d, int m,
+                               Codebooks cb, WsHeader hdr, char *__restrict__ ws, WsLayout L) {
+    float *Rc = (float *)(ws + L.R);
+    float *RT = (float *)(ws + L.RT);
+    float *ST = (float *)(ws + L.ST);
+    float *SpT = (float *)(ws + L.SpT);
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nth = (int64_t)gridDim.x * blockDim.x;
+    if (tid == 0) {
+        *(WsHeader *)(ws + L.header) = hdr;
+        *(Codebooks *)(ws + L.codebooks) = cb;
+    }
+    for (int64_t e = tid; e < (int64_t)d * d; e += nth) {
+        int i = (int)(e / d), j = (int)(e % d);
+        float v = R[e];
+        Rc[e] = v;
+        RT[(int64_t)j * d + i] = v;
+    }
+    if (m <= 0) return;
+    for (int64_t e = tid; e < (int64_t)m * d; e += nth) {
+        int a = (int)(e / d), j = (int)(e % d);
+        ST[(int64_t)j * m + a] = S[e];
+    }
+    // S' = S R^T expressed on rotated coordinates: S'[a][i] = sum_k S[a][k] R[i][k],
+    // accumulated in double and rounded once.
+    for (int64_t e = tid; e < (int64_t)m * d; e += nth) {
+        int a = (int)(e / d), i = (int)(e % d);
+        const float *sr = S + (int64_t)a * d;
+        const float *rr = R + (int64_t)i * d;
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += (double)sr[k] * (double)rr[k];
+        SpT[(int64_t)i * m + a] = (float)acc;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prepare(const tq_params *p, const Codebooks &cb, cudaStream_t s) {
+    WsLayout L = ws_layout(p->dim, p->proj_dim);
+    WsHeader h{kWsMagic, p->dim, p->bits, p->proj_dim};
+    int64_t work = (int64_t)p->dim * (p->dim > p->proj_dim ? p->dim : p->proj_dim);
+    int blocks = (int)((work + 255) / 256);
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    prepare_kernel<<<blocks, 256, 0, s>>>(p->R, p->S, p->dim, p->proj_dim, cb, h,
+                                         (char *)p->workspace, L);
+    return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,453 @@
+// tq_score.cu -- query preparation, asymmetric scores, top-k and fused decode attention.
+//
+// Scores straight from packed keys (TurboQuantProd.inner_product / asymmetric attention
+// scores; "turboquant-pytorch", nav.superapi.store, 核心 API and 常见使用模式):
+//   s = ||k|| * ( <R q, c[idx]> + rho * sqrt(pi/2)/m * <S q, 2*sign - 1> )
+// which equals <q, R^T c[idx]> + ... because R is orthogonal: the query is rotated once
+// (q_rot = R q, sq = S q) instead of dequantizing every key.
+// Attention: softmax(scale * s) over the tokens, then the weighted sum of the values'
+// centroids in the rotated domain, o_rot = sum_t a_t ||v_t|| c[vidx_t], rotated back once
+// per query (o = R^T o_rot).  Long contexts are split across CTAs (partial max, sum and
+// o_rot per split) and combined with the usual log-sum-exp rescaling.
+#include <math.h>
+
+#include "tq_common.cuh"
+#include "tq_internal.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kTile = 128;     // tokens per CTA tile (one per thread)
+constexpr int kMaxRows = 16;   // query rows handled per pass
+
+inline int rows_per_pass(int d, int m, int cap_regs) {
+    int by_smem = (int)((40 * 1024 / sizeof(float)) / (size_t)(d + m));
+    int r = kMaxRows;
+    if (by_smem < r) r = by_smem;
+    if (cap_regs < r) r = cap_regs;
+    return r < 1 ? 1 : r;
+}
+
+// ------------------------------------------------------------------ query prep
+
+__global__ void qprep_kernel(Prepared P, const float *__restrict__ q, int64_t rows,
+                             float *__restrict__ out) {
+    extern __shared__ float qs[];
+    const int d = P.d, m = P.m;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        for (int j = threadIdx.x; j < d; j += blockDim.x) qs[j] = q[row * d + j];
+        __syncthreads();
+        float *o = out + row * (d + m);
+        for (int i = threadIdx.x; i < d; i += blockDim.x) {
+            float acc = 0.f;
+            for (int j = 0; j < d; ++j) acc = fmaf(P.RT[(int64_t)j * d + i], qs[j], acc);
+            o[i] = acc;
+        }
+        for (int a = threadIdx.x; a < m; a += blockDim.x) {
+            float acc = 0.f;
+            for (int j = 0; j < d; ++j) acc = fmaf(P.ST[(int64_t)j * m + a], qs[j], acc);
+            o[d + a] = acc;
+        }
+        __syncthreads();
+    }
+}
+
+// Accumulate, for one packed key and `rch` query rows, the MSE dot <q_rot, c[idx]>
+// (acc) and the sign dot <sq, 2*sign-1> (acc2).
+template <int RM>
+__device__ __forceinline__ void key_dots(const Prepared &P, const float *cen, const float *qs,
+                                         int rch, const uint32_t *kc, const uint32_t *ks,
+                                         float *acc, float *acc2) {
+    const int d = P.d, m = P.m, beta = P.kbeta, stride = d + m;
+    for (int g = 0; g < (d >> 5); ++g) {
+        uint32_t w[4] = {0, 0, 0, 0};
+        for (int p = 0; p < beta; ++p) w[p] = kc[g * beta + p];
+        for (int l = 0; l < 32; ++l) {
+            int idx = 0;
+            for (int p = 0; p < beta; ++p) idx |= ((w[p] >> l) & 1u) << p;
+            const float c = cen[idx];
+            const int j = 32 * g + l;
+#pragma unroll
+            for (int r = 0; r < RM; ++r)
+                if (r < rch) acc[r] = fmaf(qs[r * stride + j], c, acc[r]);
+        }
+    }
+    for (int g = 0; g < (m >> 5); ++g) {
+        const uint32_t w = ks[g];
+        for (int l = 0; l < 32; ++l) {
+            const int a = 32 * g + l;
+            const bool pos = (w >> l) & 1u;
+#pragma unroll
+            for (int r = 0; r < RM; ++r)
+                if (r < rch) {
+                    const float s = qs[r * stride + d + a];
+                    acc2[r] += pos ? s : -s;
+                }
+        }
+    }
+}
+
+__device__ __forceinline__ int64_t query_row(const ScoreProblem &sp, int b, int kv, int r) {
+    const int G = sp.Hq / sp.Hkv;
+    const int g = r / sp.Nq, i = r % sp.Nq;
+    return ((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i;
+}
+
+// --------------------------------------------------------------------- scores
+
+__global__ void __launch_bounds__(kTile) scores_kernel(Prepared P, ScoreProblem sp,
+                                                       const float *__restrict__ qprep, int rpp,
+                                                       float *__restrict__ scores) {
+    extern __shared__ float qs[];
+    __shared__ float cen[kMaxLevels];
+    const int d = P.d, m = P.m, stride = d + m;
+    if (threadIdx.x < kMaxLevels) cen[threadIdx.x] = P.cb->kc[threadIdx.x];
+    const int64_t sl = blockIdx.y;
+    const int b = (int)(sl / sp.Hkv), kv = (int)(sl % sp.Hkv);
+    const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
+    const int64_t t = (int64_t)blockIdx.x * kTile + threadIdx.x;
+    const bool valid = t < sp.T;
+    const int64_t rec = sl * sp.T + t;
+    const float gamma = sqrtf(1.5707963267948966f) / (float)m;
+    const int wpk = P.kbeta * (d >> 5), spk = m >> 5;
+    float kn = 0.f, rn = 0.f;
+    if (valid) {
+        kn = f16_bits_to_f32(sp.knorm[rec]);
+        rn = f16_bits_to_f32(sp.krnorm[rec]);
+    }
+    for (int r0 = 0; r0 < rows; r0 += rpp) {
+        const int rch = min(rpp, rows - r0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < rch * stride; e += blockDim.x) {
+            const int r = e / stride, c = e % stride;
+            qs[e] = qprep[query_row(sp, b, kv, r0 + r) * stride + c];
+        }
+        __syncthreads();
+        if (valid) {
+            float acc[kMaxRows], acc2[kMaxRows];
+#pragma unroll
+            for (int r = 0; r < kMaxRows; ++r) acc[r] = acc2[r] = 0.f;
+            key_dots<kMaxRows>(P, cen, qs, rch, sp.kcodes + rec * wpk, sp.ksigns + rec * spk, acc, acc2);
+#pragma unroll
+            for (int r = 0; r < kMaxRows; ++r)
+                if (r < rch)
+                    scores[query_row(sp, b, kv, r0 + r) * sp.T + t] = kn * fmaf(rn * gamma, acc2[r], acc[r]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------- top-k
+
+struct Cand {
+    float v;
+    int32_t i;
+};
+
+__device__ __forceinline__ bool better(float va, int32_t ia, float vb, int32_t ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+constexpr int kTopkThreads = 256;
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float *__restrict__ scores, int64_t T,
+                                                            int k, int32_t *__restrict__ oidx,
+                                                            float *__restrict__ oval) {
+    const int64_t row = blockIdx.x;
+    const float *s = scores + row * T;
+    float lv[kMaxTopk];
+    int32_t li[kMaxTopk];
+    int cnt = 0;
+    for (int64_t t = threadIdx.x; t < T; t += kTopkThreads) {
+        const float v = s[t];
+        const int32_t ti = (int32_t)t;
+        if (cnt == k && !better(v, ti, lv[k - 1], li[k - 1])) continue;
+        int pos = cnt < k ? cnt : k - 1;
+        while (pos > 0 && better(v, ti, lv[pos - 1], li[pos - 1])) {
+            lv[pos] = lv[pos - 1];
+            li[pos] = li[pos - 1];
+            --pos;
+        }
+        lv[pos] = v;
+        li[pos] = ti;
+        if (cnt < k) ++cnt;
+    }
+    // k rounds of a block-wide arg-max over the heads of the per-thread sorted lists
+    __shared__ float wv[kTopkThreads / 32];
+    __shared__ int32_t wi[kTopkThreads / 32];
+    int head = 0;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int round = 0; round < k; ++round) {
+        float v = head < cnt ? lv[head] : -INFINITY;
+        int32_t i = head < cnt ? li[head] : INT32_MAX;
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(kFull, v, o);
+            const int32_t oi = __shfl_xor_sync(kFull, i, o);
+            if (better(ov, oi, v, i)) { v = ov; i = oi; }
+        }
+        if (lane == 0) { wv[warp] = v; wi[warp] = i; }
+        __syncthreads();
+        if (warp == 0) {
+            v = lane < kTopkThreads / 32 ? wv[lane] : -INFINITY;
+            i = lane < kTopkThreads / 32 ? wi[lane] : INT32_MAX;
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, v, o);
+                const int32_t oi = __shfl_xor_sync(kFull, i, o);
+                if (better(ov, oi, v, i)) { v = ov; i = oi; }
+            }
+            if (lane == 0) { wv[0] = v; wi[0] = i; oidx[row * k + round] = i; oval[row * k + round] = v; }
+        }
+        __syncthreads();
+        if (head < cnt && li[head] == wi[0]) ++head;
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ attention
+
+template <int CPT, int RM = (64 / CPT < kMaxRows ? 64 / CPT : kMaxRows)>
+__global__ void __launch_bounds__(kTile) attend_kernel(Prepared P, ScoreProblem sp,
+                                                       const float *__restrict__ qprep, int rpp,
+                                                       float scale, float *__restrict__ partials,
+                                                       int splits) {
+    extern __shared__ float smem[];
+    __shared__ float kcen[kMaxLevels], vcen[kMaxLevels];
+    __shared__ float rowM[kMaxRows], rowL[kMaxRows], rowA[kMaxRows];
+    const int d = P.d, m = P.m, stride = d + m;
+    float *qs = smem;
+    float *ps = smem + rpp * stride;
+    if (threadIdx.x < kMaxLevels) {
+        kcen[threadIdx.x] = P.cb->kc[threadIdx.x];
+        vcen[threadIdx.x] = P.cb->vc[threadIdx.x];
+    }
+    const int split = blockIdx.x;
+    const int64_t sl = blockIdx.y;
+    const int b = (int)(sl / sp.Hkv), kv = (int)(sl % sp.Hkv);
+    const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
+    const int64_t chunk = (sp.T + splits - 1) / splits;
+    const int64_t t0 = (int64_t)split * chunk;
+    const int64_t t1 = min(sp.T, t0 + chunk);
+    const float gamma = sqrtf(1.5707963267948966f) / (float)m;
+    const int wpk = P.kbeta * (d >> 5), spk = m >> 5, vwpv = P.vbeta * (d >> 5), vbeta = P.vbeta;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t rows_total = (int64_t)sp.B * sp.Hq * sp.Nq;
+
+    for (int r0 = 0; r0 < rows; r0 += rpp) {
+        const int rch = min(rpp, rows - r0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < rch * stride; e += blockDim.x) {
+            const int r = e / stride, c = e % stride;
+            qs[e] = qprep[query_row(sp, b, kv, r0 + r) * stride + c];
+        }
+        if (threadIdx.x < kMaxRows) {
+            rowM[threadIdx.x] = -INFINITY;
+            rowL[threadIdx.x] = 0.f;
+        }
+        float o[RM][CPT];
+#pragma unroll
+        for (int r = 0; r < RM; ++r)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) o[r][c] = 0.f;
+        __syncthreads();
+        for (int64_t tb = t0; tb < t1; tb += kTile) {
+            // scores of this tile, one token per thread
+            const int64_t t = tb + threadIdx.x;
+            const bool valid = t < t1;
+            {
+                float acc[RM], acc2[RM];
+#pragma unroll
+                for (int r = 0; r < RM; ++r) acc[r] = acc2[r] = 0.f;
+                float kn = 0.f, rn = 0.f;
+                if (valid) {
+                    const int64_t rec = sl * sp.T + t;
+                    kn = f16_bits_to_f32(sp.knorm[rec]);
+                    rn = f16_bits_to_f32(sp.krnorm[rec]);
+                    key_dots<RM>(P, kcen, qs, rch, sp.kcodes + rec * wpk, sp.ksigns + rec * spk, acc, acc2);
+                }
+#pragma unroll
+                for (int r = 0; r < RM; ++r)
+                    if (r < rch)
+                        ps[r * kTile + threadIdx.x] =
+                            valid ? scale * (kn * fmaf(rn * gamma, acc2[r], acc[r])) : -INFINITY;
+            }
+            __syncthreads();
+            // online softmax bookkeeping: one warp per row
+            for (int r = warp; r < rch; r += kTile / 32) {
+                float mx = -INFINITY;
+                for (int q = lane; q < kTile; q += 32) mx = fmaxf(mx, ps[r * kTile + q]);
+                mx = warp_max(mx);
+                const float oldM = rowM[r];
+                const float newM = fmaxf(oldM, mx);
+                const float alpha = (oldM == -INFINITY) ? 0.f : expf(oldM - newM);
+                float sum = 0.f;
+                for (int q = lane; q < kTile; q += 32) {
+                    const float sv = ps[r * kTile + q];
+                    const float e = (sv == -INFINITY) ? 0.f : expf(sv - newM);
+                    ps[r * kTile + q] = e;
+                    sum += e;
+                }
+                sum = warp_sum(sum);
+                if (lane == 0) {
+                    rowL[r] = rowL[r] * alpha + sum;
+                    rowM[r] = newM;
+                    rowA[r] = alpha;
+                }
+            }
+            __syncthreads();
+            // weighted value sum in the rotated domain; thread owns coordinates tid + 128c
+#pragma unroll
+            for (int r = 0; r < RM; ++r)
+                if (r < rch) {
+                    const float a = rowA[r];
+#pragma unroll
+                    for (int c = 0; c < CPT; ++c) o[r][c] *= a;
+                }
+            const int ntok = (int)min((int64_t)kTile, t1 - tb);
+            for (int tt = 0; tt < ntok; ++tt) {
+                const int64_t rec = sl * sp.T + tb + tt;
+                const float vn = f16_bits_to_f32(sp.vnorm[rec]);
+                const uint32_t *vw = sp.vcodes + rec * vwpv;
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    const int j = threadIdx.x + kTile * c;
+                    if (j < d) {
+                        const int g = j >> 5, l = j & 31;
+                        int idx = 0;
+                        for (int p = 0; p < vbeta; ++p) idx |= ((vw[g * vbeta + p] >> l) & 1u) << p;
+                        const float w = vn * vcen[idx];
+#pragma unroll
+                        for (int r = 0; r < RM; ++r)
+                            if (r < rch) o[r][c] = fmaf(ps[r * kTile + tt], w, o[r][c]);
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        // partials[row][split] = (M, L, o_rot[d])
+#pragma unroll
+        for (int r = 0; r < RM; ++r)
+            if (r < rch) {
+                float *pp = partials + (query_row(sp, b, kv, r0 + r) * splits + split) * (int64_t)(d + 2);
+                if (threadIdx.x == 0) {
+                    pp[0] = rowM[r];
+                    pp[1] = rowL[r];
+                }
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    const int j = threadIdx.x + kTile * c;
+                    if (j < d) pp[2 + j] = o[r][c];
+                }
+            }
+    }
+    (void)rows_total;
+}
+
+__global__ void attend_combine_kernel(Prepared P, int64_t rows, int splits,
+                                      const float *__restrict__ partials, float *__restrict__ out) {
+    extern __shared__ float orot[];
+    const int d = P.d;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const float *pp = partials + row * splits * (int64_t)(d + 2);
+        float M = -INFINITY;
+        for (int s = 0; s < splits; ++s) M = fmaxf(M, pp[(int64_t)s * (d + 2)]);
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float acc = 0.f, L = 0.f;
+            for (int s = 0; s < splits; ++s) {
+                const float *ps = pp + (int64_t)s * (d + 2);
+                const float w = (ps[0] == -INFINITY) ? 0.f : expf(ps[0] - M);
+                acc = fmaf(w, ps[2 + j], acc);
+                L = fmaf(w, ps[1], L);
+            }
+            orot[j] = acc / L;
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float acc = 0.f;
+            for (int i = 0; i < d; ++i) acc = fmaf(P.R[(int64_t)i * d + j], orot[i], acc);
+            out[row * d + j] = acc;
+        }
+        __syncthreads();
+    }
+}
+
+int attend_splits(const ScoreProblem &sp) {
+    const int64_t slices = (int64_t)sp.B * sp.Hkv;
+    int64_t want = (148 * 4 + slices - 1) / slices;
+    int64_t cap = (sp.T + 255) / 256;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    return (int)want;
+}
+
+}  // namespace
+
+size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp) {
+    return align_up(sizeof(float) * (size_t)sp.B * sp.Hq * sp.Nq * (P.d + P.m), 256);
+}
+
+size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int *splits_out) {
+    int splits = attend_splits(sp);
+    if (splits_out) *splits_out = splits;
+    return align_up(sizeof(float) * (size_t)sp.B * sp.Hq * sp.Nq * splits * (P.d + 2), 256);
+}
+
+size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk) {
+    (void)P;
+    (void)topk;
+    return align_up(sizeof(float) * (size_t)sp.B * sp.Hq * sp.Nq * (size_t)sp.T, 256);
+}
+
+cudaError_t launch_qprep(const Prepared &P, const ScoreProblem &sp, float *qprep, cudaStream_t s) {
+    const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
+    int blocks = (int)(rows < 148 * 8 ? rows : 148 * 8);
+    qprep_kernel<<<blocks, 128, sizeof(float) * P.d, s>>>(P, sp.q, rows, qprep);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scores(const Prepared &P, const ScoreProblem &sp, const float *qprep, float *scores,
+                          cudaStream_t s) {
+    const int rpp = rows_per_pass(P.d, P.m, kMaxRows);
+    const size_t smem = sizeof(float) * (size_t)rpp * (P.d + P.m);
+    dim3 grid((unsigned)((sp.T + kTile - 1) / kTile), (unsigned)(sp.B * sp.Hkv));
+    cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    scores_kernel<<<grid, kTile, smem, s>>>(P, sp, qprep, rpp, scores);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const ScoreProblem &sp, const float *scores, int topk, int32_t *idx, float *val,
+                        cudaStream_t s) {
+    const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
+    topk_kernel<<<(unsigned)rows, kTopkThreads, 0, s>>>(scores, sp.T, topk, idx, val);
+    return cudaGetLastError();
+}
+
+template <int CPT>
+static cudaError_t launch_attend_cpt(const Prepared &P, const ScoreProblem &sp, const float *qprep,
+                                     float scale, float *partials, int splits, cudaStream_t s) {
+    const int rpp = rows_per_pass(P.d, P.m, 64 / CPT < kMaxRows ? 64 / CPT : kMaxRows);
+    const size_t smem = sizeof(float) * ((size_t)rpp * (P.d + P.m) + (size_t)rpp * kTile);
+    cudaFuncSetAttribute(attend_kernel<CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid((unsigned)splits, (unsigned)(sp.B * sp.Hkv));
+    attend_kernel<CPT><<<grid, kTile, smem, s>>>(P, sp, qprep, rpp, scale, partials, splits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale,
+                          float *partials, int splits, float *out, cudaStream_t s) {
+    cudaError_t e;
+    const int cpt = (P.d + kTile - 1) / kTile;
+    switch (cpt) {
+        case 1: e = launch_attend_cpt<1>(P, sp, qprep, scale, partials, splits, s); break;
+        case 2: e = launch_attend_cpt<2>(P, sp, qprep, scale, partials, splits, s); break;
+        case 4: e = launch_attend_cpt<4>(P, sp, qprep, scale, partials, splits, s); break;
+        case 8: e = launch_attend_cpt<8>(P, sp, qprep, scale, partials, splits, s); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
+    int blocks = (int)(rows < 148 * 8 ? rows : 148 * 8);
+    attend_combine_kernel<<<blocks, 128, sizeof(float) * P.d, s>>>(P, rows, splits, partials, out);
+    return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,233 @@
+"""GPU parity: the CUDA path through the C ABI against the oracle, element by element, on
+seeded inputs that span several tiles, ragged tails and the degenerate cases."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from kv_cache_vector_compress_b200 import synth
+
+from .parity import (as_u16, as_u32, check_close, check_codes, check_f16_close, check_signs, check_topk)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tq():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from kv_cache_vector_compress_b200 import tq as _tq  # raises if libtq.so is missing
+    return _tq
+
+
+def _params(tq, R, S, bits, m):
+    import torch
+    d = R.shape[0]
+    Rt = torch.from_numpy(R).cuda()
+    St = torch.from_numpy(S).cuda() if S is not None else None
+    return tq.Params(d, bits, m, Rt, St)
+
+
+def _compress_both(tq, x, R, S, bits, is_key):
+    """GPU and oracle compression of the same rows; asserts the parity rules and returns both."""
+    import torch
+    d = R.shape[0]
+    m = S.shape[0] if S is not None else 0
+    p = _params(tq, R, S, bits, m)
+    xt = torch.from_numpy(x).cuda()
+    ora = oracle.compress(x, R, S, bits, is_key=is_key, want_y=True, want_p=is_key)
+    if is_key:
+        codes, signs, norm, rnorm = tq.tq_compress_keys(p, xt)
+    else:
+        codes, norm = tq.tq_compress_values(p, xt)
+    torch.cuda.synchronize()
+    beta = bits - 1 if is_key else bits
+    bnd, _ = oracle.codebook_f32(d, beta)
+    rows = check_codes(codes, ora["codes"], ora["y32"], bnd, d, beta)
+    check_f16_close(norm, ora["norm"], what="norm")
+    gpu = {"codes": codes, "norm": norm}
+    if is_key:
+        check_signs(signs, ora["signs"], ora["p32"], m, exempt_rows=rows)
+        check_f16_close(rnorm, ora["rnorm"], exempt_rows=rows, what="rnorm")
+        gpu.update(signs=signs, rnorm=rnorm)
+    return gpu, ora, rows, p
+
+
+# ------------------------------------------------------------------ compress
+
+def test_compress_workload1(tq):
+    w = synth.workload1()
+    _, _, rk, _ = _compress_both(tq, w["K"], w["R"], w["S"], 3, True)
+    _, _, rv, _ = _compress_both(tq, w["V"], w["R"], None, 3, False)
+    assert len(rk) <= 2 and len(rv) <= 2
+
+
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
+@pytest.mark.parametrize("n", [1, 31, 33, 257])
+@pytest.mark.parametrize("f16", [True, False])
+def test_compress_shapes(tq, d, n, f16):
+    R = synth.rotation(d, 1000 + d)
+    S = synth.gaussian(d // 2, d, 2000 + d)
+    x = synth.gaussian(n, d, 3000 + n + d)
+    x = x.astype(np.float16) if f16 else x
+    for bits in (2, 3, 4):
+        _compress_both(tq, x, R, S, bits, True)
+    for bits in (1, 2, 3, 4):
+        _compress_both(tq, x, R, None, bits, False)
+
+
+def test_compress_zero_and_outlier_rows(tq):
+    d = 128
+    R = synth.rotation(d, 11)
+    S = synth.gaussian(64, d, 12)
+    x = synth.channel_scaled_f16(96, d, 13, 14, 3)
+    x[5] = 0
+    x[40, :3] = np.float16(60000.0)  # near the top of the fp16 range
+    gk, ok, _, _ = _compress_both(tq, x, R, S, 3, True)
+    gv, ov, _, _ = _compress_both(tq, x, R, None, 3, False)
+    assert as_u16(gk["norm"])[5] == 0 and as_u16(gv["norm"])[5] == 0
+
+
+def test_compress_large_projection(tq):
+    d, m = 64, 256
+    R = synth.rotation(d, 21)
+    S = synth.gaussian(m, d, 22)
+    x = synth.gaussian(300, d, 23)
+    _compress_both(tq, x, R, S, 2, True)
+
+
+# -------------------------------------------------------------------- scores
+
+def _oracle_cache(seed, d, m, bits, B, Hkv, T, f16=True):
+    R = synth.rotation(d, seed)
+    S = synth.gaussian(m, d, seed + 1)
+    K = synth.gaussian(B * Hkv * T, d, seed + 2)
+    V = synth.gaussian(B * Hkv * T, d, seed + 3)
+    if f16:
+        K, V = K.astype(np.float16), V.astype(np.float16)
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    v = oracle.compress(V, R, None, bits, is_key=False)
+    return R, S, k, v
+
+
+def _to_dev(k, v=None):
+    import torch
+    kk = (torch.from_numpy(k["codes"].view(np.int32)).cuda(), torch.from_numpy(k["signs"].view(np.int32)).cuda(),
+          torch.from_numpy(k["norm"].view(np.float16)).cuda(), torch.from_numpy(k["rnorm"].view(np.float16)).cuda())
+    if v is None:
+        return kk
+    vv = (torch.from_numpy(v["codes"].view(np.int32)).cuda(), torch.from_numpy(v["norm"].view(np.float16)).cuda())
+    return kk, vv
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(d=128, m=64, bits=3, B=1, Hkv=1, G=1, Nq=16, T=4096),   # workload 1 shape
+    dict(d=64, m=32, bits=2, B=2, Hkv=2, G=4, Nq=1, T=300),      # GQA, ragged tail
+    dict(d=128, m=64, bits=4, B=1, Hkv=1, G=1, Nq=20, T=129),    # more rows than one pass
+    dict(d=256, m=128, bits=2, B=1, Hkv=2, G=2, Nq=2, T=77),     # wide head, 1-bit keys
+    dict(d=32, m=32, bits=3, B=3, Hkv=1, G=1, Nq=1, T=1),        # single token
+])
+def test_scores_on_oracle_cache(tq, cfg):
+    import torch
+    c = cfg
+    R, S, k, _ = _oracle_cache(100 + c["d"] + c["T"], c["d"], c["m"], c["bits"], c["B"], c["Hkv"], c["T"])
+    Hq = c["Hkv"] * c["G"]
+    q = synth.gaussian(c["B"] * Hq * c["Nq"], c["d"], 7).reshape(c["B"], Hq, c["Nq"], c["d"])
+    ora = oracle.scores(q, R, S, c["bits"], c["B"], Hq, c["Hkv"], c["Nq"], c["T"],
+                        k["codes"], k["signs"], k["norm"], k["rnorm"])
+    p = _params(tq, R, S, c["bits"], c["m"])
+    s, _, _ = tq.tq_scores(p, torch.from_numpy(q).cuda(), _to_dev(k), c["Hkv"], c["T"])
+    torch.cuda.synchronize()
+    check_close(s, ora, "scores")
+
+
+@pytest.mark.parametrize("k_", [1, 10, 64])
+def test_scores_topk(tq, k_):
+    import torch
+    d, m, bits, T, Nq = 64, 32, 3, 3000, 18
+    R, S, k, _ = _oracle_cache(500 + k_, d, m, bits, 1, 1, T, f16=False)
+    q = synth.gaussian(Nq, d, 8).reshape(1, 1, Nq, d)
+    ora = oracle.scores(q, R, S, bits, 1, 1, 1, Nq, T, k["codes"], k["signs"], k["norm"], k["rnorm"])
+    p = _params(tq, R, S, bits, m)
+    for want_scores in (True, False):
+        s, ti, tv = tq.tq_scores(p, torch.from_numpy(q).cuda(), _to_dev(k), 1, T, want_scores=want_scores,
+                                 topk=k_)
+        torch.cuda.synchronize()
+        if want_scores:
+            check_close(s, ora, "scores")
+        for r in range(Nq):
+            check_topk(ti[0, 0, r].cpu().numpy(), tv[0, 0, r].cpu().numpy(), ora[0, 0, r], k_, f"row {r}")
+
+
+def test_scores_topk_exact_ties(tq):
+    # identical keys give identical scores: ties resolve to the smaller token index
+    import torch
+    d, m, bits, T = 32, 32, 2, 500
+    R = synth.rotation(d, 1)
+    S = synth.gaussian(m, d, 2)
+    K = np.repeat(synth.gaussian(5, d, 3), 100, axis=0)
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    q = synth.gaussian(1, d, 4).reshape(1, 1, 1, d)
+    p = _params(tq, R, S, bits, m)
+    _, ti, tv = tq.tq_scores(p, torch.from_numpy(q).cuda(), _to_dev(k), 1, T, want_scores=False, topk=10)
+    ora = oracle.scores(q, R, S, bits, 1, 1, 1, 1, T, k["codes"], k["signs"], k["norm"], k["rnorm"])[0, 0, 0]
+    best = int(np.argmax(ora[::100]))
+    np.testing.assert_array_equal(ti[0, 0, 0].cpu().numpy(), np.arange(100 * best, 100 * best + 10))
+
+
+# -------------------------------------------------------------------- attend
+
+@pytest.mark.parametrize("cfg", [
+    dict(d=128, m=64, bits=3, B=1, Hkv=1, G=1, Nq=16, T=4096),
+    dict(d=128, m=64, bits=3, B=2, Hkv=2, G=4, Nq=1, T=1000),
+    dict(d=64, m=32, bits=2, B=1, Hkv=1, G=2, Nq=10, T=1),
+    dict(d=64, m=32, bits=4, B=1, Hkv=2, G=1, Nq=17, T=129),
+    dict(d=256, m=128, bits=2, B=1, Hkv=1, G=4, Nq=1, T=3000),
+    dict(d=256, m=128, bits=4, B=1, Hkv=1, G=4, Nq=1, T=513),
+    dict(d=32, m=32, bits=1 + 1, B=1, Hkv=1, G=1, Nq=1, T=127),
+])
+def test_attend_on_oracle_cache(tq, cfg):
+    import torch
+    c = cfg
+    R, S, k, v = _oracle_cache(300 + c["d"] + c["T"], c["d"], c["m"], c["bits"], c["B"], c["Hkv"], c["T"])
+    Hq = c["Hkv"] * c["G"]
+    q = synth.gaussian(c["B"] * Hq * c["Nq"], c["d"], 9).reshape(c["B"], Hq, c["Nq"], c["d"])
+    ora = oracle.attend(q, R, S, c["bits"], c["B"], Hq, c["Hkv"], c["Nq"], c["T"], k["codes"], k["signs"],
+                        k["norm"], k["rnorm"], v["codes"], v["norm"])
+    p = _params(tq, R, S, c["bits"], c["m"])
+    kk, vv = _to_dev(k, v)
+    out = tq.tq_attend(p, torch.from_numpy(q).cuda(), kk, vv, c["Hkv"], c["T"])
+    torch.cuda.synchronize()
+    check_close(out, ora, "attend")
+    # an explicit temperature
+    ora2 = oracle.attend(q, R, S, c["bits"], c["B"], Hq, c["Hkv"], c["Nq"], c["T"], k["codes"], k["signs"],
+                         k["norm"], k["rnorm"], v["codes"], v["norm"], scale=0.02)
+    out2 = tq.tq_attend(p, torch.from_numpy(q).cuda(), kk, vv, c["Hkv"], c["T"], scale=0.02)
+    torch.cuda.synchronize()
+    check_close(out2, ora2, "attend scale=0.02")
+
+
+def test_end_to_end_workload1(tq):
+    """Compress with the GPU, attend with the GPU; oracle does the same from the same inputs."""
+    import torch
+    w = synth.workload1()
+    R, S = w["R"], w["S"]
+    p = _params(tq, R, S, 3, 64)
+    kt = tq.tq_compress_keys(p, torch.from_numpy(w["K"]).cuda())
+    vt = tq.tq_compress_values(p, torch.from_numpy(w["V"]).cuda())
+    q = torch.from_numpy(w["Q"]).cuda()
+    out = tq.tq_attend(p, q, kt, vt, 1, 4096)
+    s, _, _ = tq.tq_scores(p, q, kt, 1, 4096)
+    torch.cuda.synchronize()
+    k = oracle.compress(w["K"], R, S, 3, is_key=True)
+    v = oracle.compress(w["V"], R, None, 3, is_key=False)
+    ora_out = oracle.attend(w["Q"], R, S, 3, 1, 1, 1, 16, 4096, k["codes"], k["signs"], k["norm"], k["rnorm"],
+                            v["codes"], v["norm"])
+    check_close(out, ora_out, "end-to-end attend")
+    ora_s = oracle.scores(w["Q"], R, S, 3, 1, 1, 1, 16, 4096, k["codes"], k["signs"], k["norm"], k["rnorm"])
+    # keys whose packed records are identical must score within tolerance
+    same = ((as_u32(kt[0]) == k["codes"]).all(1) & (as_u32(kt[1]) == k["signs"]).all(1)
+            & (as_u16(kt[2]) == k["norm"]) & (as_u16(kt[3]) == k["rnorm"]))
+    assert same.mean() > 0.999
+    check_close(s[0, 0][:, torch.from_numpy(same).cuda()], ora_s[0, 0][:, same], "end-to-end scores")
