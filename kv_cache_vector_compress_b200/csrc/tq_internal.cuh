@@ -32,8 +32,25 @@ struct WsLayout {
     size_t RT;         // fp32 [d, d]      R transposed
     size_t ST;         // fp32 [d, m]      S transposed
     size_t SpT;        // fp32 [d, m]      (S R^T) transposed
+    size_t Rsw;        // fp16 hi | lo of R * 2^kRScaleLog2, tensor-core operand layout
+    size_t Ssw;        // fp16 hi | lo of (S R^T) * 2^kSScaleLog2, same layout
     size_t total;
 };
+
+// Split-precision scales: R (entries <= 1) and S' = S R^T (entries ~N(0,1)) are scaled
+// by a power of two before the fp16 hi/lo split so that the lo parts stay normal numbers.
+constexpr int kRScaleLog2 = 8;
+constexpr int kSScaleLog2 = 4;
+
+// Byte offset of element (r, k) of a K-major fp16 operand with `rows` rows in the
+// 128-byte-swizzled layout the tensor cores read: K is cut into blocks of 64 elements
+// (128 bytes); each block holds `rows` rows of 128 bytes; the 16-byte chunk index of a
+// row is XORed with (row mod 8).  Blocks start on 1024-byte boundaries when rows % 8 == 0.
+__host__ __device__ inline size_t sw128_offset(int rows, int r, int k) {
+    const int kb = k >> 6, kk = k & 63;
+    const int chunk = (kk * 2) >> 4, within = (kk * 2) & 15;
+    return (size_t)kb * rows * 128 + (size_t)r * 128 + (size_t)(((chunk ^ (r & 7)) << 4) + within);
+}
 
 struct WsHeader {
     uint32_t magic;
@@ -56,7 +73,11 @@ inline WsLayout ws_layout(int d, int m) {
     L.ST = o;
     o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 256);
     L.SpT = o;
-    o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 256);
+    o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 1024);
+    L.Rsw = o;
+    o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * d, 1024);
+    L.Ssw = o;
+    o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * (m > 0 ? m : 1), 1024);
     L.total = o;
     return L;
 }
@@ -66,6 +87,7 @@ struct Prepared {
     int d, m, kbeta, vbeta;
     const Codebooks *cb;
     const float *R, *RT, *ST, *SpT;
+    const uint16_t *Rsw, *Ssw;
 };
 
 inline Prepared prepared_view(const tq_params *p) {
@@ -81,6 +103,8 @@ inline Prepared prepared_view(const tq_params *p) {
     v.RT = (const float *)(w + L.RT);
     v.ST = (const float *)(w + L.ST);
     v.SpT = (const float *)(w + L.SpT);
+    v.Rsw = (const uint16_t *)(w + L.Rsw);
+    v.Ssw = (const uint16_t *)(w + L.Ssw);
     return v;
 }
 
@@ -89,6 +113,10 @@ int lloyd_max_gaussian(int dim, int bits, double *bounds, double *cents);
 
 // Kernel launchers (tq_*.cu).  All return a cudaError_t from cudaGetLastError.
 cudaError_t launch_prepare(const tq_params *p, const Codebooks &cb, cudaStream_t s);
+bool compress_tc_supported(const Prepared &P, bool is_key, bool x_f16);
+cudaError_t launch_compress_tc(const Prepared &P, bool is_key, const void *x, int64_t n, uint32_t *codes,
+                               uint32_t *signs, uint16_t *norm, uint16_t *rnorm, int32_t *dev_status,
+                               cudaStream_t s);
 cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
                             uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
                             int32_t *dev_status, cudaStream_t s);

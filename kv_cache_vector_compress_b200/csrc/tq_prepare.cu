@@ -17,11 +17,20 @@ __global__ void prepare_kernel(const float *__restrict__ R, const float *__restr
         *(WsHeader *)(ws + L.header) = hdr;
         *(Codebooks *)(ws + L.codebooks) = cb;
     }
+    uint16_t *Rhi = (uint16_t *)(ws + L.Rsw);
+    uint16_t *Rlo = Rhi + (size_t)d * d;
     for (int64_t e = tid; e < (int64_t)d * d; e += nth) {
         int i = (int)(e / d), j = (int)(e % d);
         float v = R[e];
         Rc[e] = v;
         RT[(int64_t)j * d + i] = v;
+        // split operand: R * 2^s = hi + lo, both fp16, row i = output coordinate, k = j
+        const float sv = v * (float)(1 << kRScaleLog2);
+        const __half hi = __float2half_rn(sv);
+        const __half lo = __float2half_rn(sv - __half2float(hi));
+        const size_t off = sw128_offset(d, i, j) / 2;
+        Rhi[off] = __half_as_ushort(hi);
+        Rlo[off] = __half_as_ushort(lo);
     }
     if (m <= 0) return;
     for (int64_t e = tid; e < (int64_t)m * d; e += nth) {
@@ -37,6 +46,15 @@ __global__ void prepare_kernel(const float *__restrict__ R, const float *__restr
         double acc = 0.0;
         for (int k = 0; k < d; ++k) acc += (double)sr[k] * (double)rr[k];
         SpT[(int64_t)i * m + a] = (float)acc;
+        // split operand of S' * 2^s: row a = projection index, k = i (rotated coordinate)
+        const double sv = acc * (double)(1 << kSScaleLog2);
+        const __half hi = __double2half(sv);
+        const __half lo = __float2half_rn((float)(sv - (double)__half2float(hi)));
+        uint16_t *Shi = (uint16_t *)(ws + L.Ssw);
+        uint16_t *Slo = Shi + (size_t)m * d;
+        const size_t off = sw128_offset(m, a, i) / 2;
+        Shi[off] = __half_as_ushort(hi);
+        Slo[off] = __half_as_ushort(lo);
     }
 }
 

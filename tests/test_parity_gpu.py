@@ -68,7 +68,7 @@ def test_compress_workload1(tq):
 @pytest.mark.parametrize("f16", [True, False])
 def test_compress_shapes(tq, d, n, f16):
     R = synth.rotation(d, 1000 + d)
-    S = synth.gaussian(d // 2, d, 2000 + d)
+    S = synth.gaussian(max(32, d // 2), d, 2000 + d)
     x = synth.gaussian(n, d, 3000 + n + d)
     x = x.astype(np.float16) if f16 else x
     for bits in (2, 3, 4):
