@@ -198,6 +198,8 @@ def run_tq(args):
     from kv_cache_vector_compress_b200 import synth, tq
 
     w = dict(W3)
+    if args.batch:
+        w["B"] = args.batch
     d, m, bits = w["d"], w["m"], w["bits"]
     B, Hq, Hkv, Nq, T = w["B"], w["Hq"], w["Hkv"], w["Nq"], w["T"]
     n = B * Hkv * T
@@ -324,7 +326,7 @@ def run_tq(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD_NAME, "parallelism": f"dp{world} (independent batches)", **w,
-                       "l2": "inputs larger than L2 (4.3 GB of fp16 K/V read per step)"},
+                       "l2": f"inputs larger than L2 ({2 * n * d * 2 / 1e9:.2f} GB of fp16 K/V read per step)"},
             "breakdown": breakdown,
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / pk["hbm_gbs"], "traffic": traffic, "peak_source": pk["source"]},
@@ -350,6 +352,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's 32)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -191,7 +191,12 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     float *sbuf = scores;
     if (!sbuf) sbuf = (float *)((char *)scratch + qprep_bytes(P, sp));
     cudaError_t e = launch_qprep(P, sp, qprep, s);
-    if (e == cudaSuccess) e = launch_scores(P, sp, qprep, sbuf, s);
+    if (e == cudaSuccess) {
+        if (decode_mma_supported(P, sp, false))
+            e = launch_decode_mma(P, sp, qprep, 1.0f, sbuf, decode_mma_splits(sp), false, s);
+        else
+            e = launch_scores(P, sp, qprep, sbuf, s);
+    }
     if (e == cudaSuccess && topk > 0) e = launch_topk(sp, sbuf, topk, topk_idx, topk_val, s);
     return from_cuda(e);
 }
@@ -202,7 +207,8 @@ size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int N
     Prepared P = prepared_view(p);
     ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                    nullptr);
-    return qprep_bytes(P, sp) + attend_partials_bytes(P, sp, nullptr);
+    const AttendPlan plan = plan_attend(P, sp);
+    return qprep_bytes(P, sp) + attend_partials_bytes(P, sp, plan.splits);
 }
 
 tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
@@ -225,11 +231,17 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     if (scale <= 0.f) scale = 1.0f / sqrtf((float)p->dim);
     cudaStream_t s = (cudaStream_t)stream;
     float *qprep = (float *)scratch;
-    int splits = 1;
-    attend_partials_bytes(P, sp, &splits);
+    const AttendPlan plan = plan_attend(P, sp);
     float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
     cudaError_t e = launch_qprep(P, sp, qprep, s);
-    if (e == cudaSuccess) e = launch_attend(P, sp, qprep, scale, partials, splits, out, s);
+    if (e == cudaSuccess) {
+        if (plan.mma) {
+            e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
+            if (e == cudaSuccess) e = launch_attend_combine(P, sp, partials, plan.splits, out, s);
+        } else {
+            e = launch_attend(P, sp, qprep, scale, partials, plan.splits, out, s);
+        }
+    }
     return from_cuda(e);
 }
 

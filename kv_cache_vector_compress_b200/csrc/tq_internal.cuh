@@ -132,7 +132,26 @@ struct ScoreProblem {
 };
 
 size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp);
-size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int *splits_out);
+int attend_splits(const ScoreProblem &sp);
+size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int splits);
+cudaError_t launch_attend_combine(const Prepared &P, const ScoreProblem &sp, const float *partials, int splits,
+                                  float *out, cudaStream_t s);
+bool decode_mma_supported(const Prepared &P, const ScoreProblem &sp, bool attend);
+int decode_mma_splits(const ScoreProblem &sp);
+cudaError_t launch_decode_mma(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale,
+                              float *out, int splits, bool attend, cudaStream_t s);
+
+// Which attention kernel a problem uses and how many context splits it takes.
+struct AttendPlan {
+    bool mma;
+    int splits;
+};
+inline AttendPlan plan_attend(const Prepared &P, const ScoreProblem &sp) {
+    AttendPlan a;
+    a.mma = decode_mma_supported(P, sp, true);
+    a.splits = a.mma ? decode_mma_splits(sp) : attend_splits(sp);
+    return a;
+}
 size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
 
 cudaError_t launch_qprep(const Prepared &P, const ScoreProblem &sp, float *qprep, cudaStream_t s);

@@ -370,6 +370,8 @@ __global__ void attend_combine_kernel(Prepared P, int64_t rows, int splits,
     }
 }
 
+}  // namespace
+
 int attend_splits(const ScoreProblem &sp) {
     const int64_t slices = (int64_t)sp.B * sp.Hkv;
     int64_t want = (148 * 4 + slices - 1) / slices;
@@ -379,15 +381,11 @@ int attend_splits(const ScoreProblem &sp) {
     return (int)want;
 }
 
-}  // namespace
-
 size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp) {
     return align_up(sizeof(float) * (size_t)sp.B * sp.Hq * sp.Nq * (P.d + P.m), 256);
 }
 
-size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int *splits_out) {
-    int splits = attend_splits(sp);
-    if (splits_out) *splits_out = splits;
+size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int splits) {
     return align_up(sizeof(float) * (size_t)sp.B * sp.Hq * sp.Nq * splits * (P.d + 2), 256);
 }
 
@@ -444,6 +442,11 @@ cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
+    return launch_attend_combine(P, sp, partials, splits, out, s);
+}
+
+cudaError_t launch_attend_combine(const Prepared &P, const ScoreProblem &sp, const float *partials, int splits,
+                                  float *out, cudaStream_t s) {
     const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
     int blocks = (int)(rows < 148 * 8 ? rows : 148 * 8);
     attend_combine_kernel<<<blocks, 128, sizeof(float) * P.d, s>>>(P, rows, splits, partials, out);
