@@ -109,7 +109,9 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     constexpr int KSTEP = D / 16;
     constexpr int KWPT = KB * G32;
     constexpr int VWPT = VB * G32;
-    constexpr bool SPLIT = !ATTEND;
+    // Scores are always carried at split precision: with large key norms (outlier channels) a
+    // single fp16 product moves the softmax logits by more than the output tolerance allows.
+    constexpr bool SPLIT = true;
     constexpr int MSTEP = KSTEP / 2;  // proj_dim = head_dim / 2
     const int m = P.m;
     constexpr int SW = MSTEP / 2;
@@ -488,15 +490,16 @@ cudaError_t launch_dm(const Prepared &P, const ScoreProblem &sp, const float *qp
 template <int D, bool ATTEND>
 cudaError_t launch_dm_bits(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale, float *out,
                            int splits, cudaStream_t s) {
-    const int kb = P.kbeta, vb = ATTEND ? P.vbeta : 1;
-#define TQ_DM_CASE(K, V) \
-    if (kb == K && vb == V) return launch_dm<D, K, V, ATTEND>(P, sp, qprep, scale, out, splits, s);
-    TQ_DM_CASE(1, 1)
-    TQ_DM_CASE(1, 2)
-    TQ_DM_CASE(2, 2)
-    TQ_DM_CASE(2, 3)
-    TQ_DM_CASE(3, 3)
-#undef TQ_DM_CASE
+    const int kb = P.kbeta, vb = P.vbeta;
+    if constexpr (ATTEND) {
+        if (kb == 1 && vb == 2) return launch_dm<D, 1, 2, true>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 2 && vb == 3) return launch_dm<D, 2, 3, true>(P, sp, qprep, scale, out, splits, s);
+    } else {
+        // scores only: the value bit width is irrelevant
+        if (kb == 1) return launch_dm<D, 1, 1, false>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 2) return launch_dm<D, 2, 1, false>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 3) return launch_dm<D, 3, 1, false>(P, sp, qprep, scale, out, splits, s);
+    }
     return cudaErrorInvalidValue;
 }
 
