@@ -25,8 +25,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileRows = 128;
-constexpr int kThreads = 320;  // 10 warps
-constexpr int kEpiWarp0 = 2;
+constexpr int kThreads = 384;  // 12 warps
+constexpr int kEpiWarp0 = 2;   // warps 2..9: epilogue (two groups of four)
+constexpr int kNormWarp0 = 10; // warps 10..11: row norms of the input tiles
 constexpr float kEScale = 1024.f;  // residual scale before the fp16 hi/lo split
 
 struct TcSmem {
@@ -53,12 +54,60 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int m, bool is_key) {
     L.bars = o;
     o += 256;
     L.misc = o;
-    o += 512;
+    o += 2048;
     L.total = o;
     return L;
 }
 
-enum BarIdx { kOpnd = 0, kFull = 1, kEmpty = 5, kRotFull = 9, kEReady = 11, kProjFull = 13, kTmemEmpty = 15 };
+enum BarIdx {
+    kOpnd = 0,
+    kFull = 1,
+    kEmpty = 5,
+    kRotFull = 9,
+    kEReady = 11,
+    kProjFull = 13,
+    kTmemEmpty = 15,
+    kNormReady = 17
+};
+
+// Code of y against ascending boundaries b[0..2^BETA-2] (#{k : b[k] < y}) by a binary
+// search whose thresholds are selected from registers.
+template <int BETA>
+__device__ __forceinline__ uint32_t bucket_tree(float y, const float (&b)[16]) {
+    if constexpr (BETA == 1) {
+        return y > b[0] ? 1u : 0u;
+    } else if constexpr (BETA == 2) {
+        const bool t1 = y > b[1];
+        const bool t0 = y > (t1 ? b[2] : b[0]);
+        return (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+    } else if constexpr (BETA == 3) {
+        const bool t2 = y > b[3];
+        const bool t1 = y > (t2 ? b[5] : b[1]);
+        const float thr = t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]);
+        const bool t0 = y > thr;
+        return (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+    } else {
+        const bool t3 = y > b[7];
+        const bool t2 = y > (t3 ? b[11] : b[3]);
+        const bool t1 = y > (t3 ? (t2 ? b[13] : b[9]) : (t2 ? b[5] : b[1]));
+        const float thr = t3 ? (t2 ? (t1 ? b[14] : b[12]) : (t1 ? b[10] : b[8]))
+                             : (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]));
+        const bool t0 = y > thr;
+        return (t3 ? 8u : 0u) | (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+    }
+}
+
+// v[idx] for a register array, as a tree of selects.
+template <int N>
+__device__ __forceinline__ float mux(const float *v, uint32_t idx) {
+    if constexpr (N == 1) {
+        return v[0];
+    } else {
+        const float lo = mux<N / 2>(v, idx);
+        const float hi = mux<N / 2>(v + N / 2, idx);
+        return (idx & (N / 2)) ? hi : lo;
+    }
+}
 
 template <int D, bool IS_KEY, int BETA>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -81,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *cen_s = bnd_s + kMaxLevels;
     uint32_t *tmem_s = (uint32_t *)(cen_s + kMaxLevels);
     volatile int *abort_s = (volatile int *)(tmem_s + 1);
+    float *norm_s = (float *)(sm + L.misc + 256);  // [2 slots][128 rows] squared norms
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
@@ -90,13 +140,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars[kOpnd], 1);
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars[kFull + s], 1);
-            mbar_init(&bars[kEmpty + s], 1);
+            mbar_init(&bars[kEmpty + s], 3);  // MMA commit + the two norm warps
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[kRotFull + s], 1);
             mbar_init(&bars[kEReady + s], 4);
             mbar_init(&bars[kProjFull + s], 1);
             mbar_init(&bars[kTmemEmpty + s], 4);
+            mbar_init(&bars[kNormReady + s], 2);
         }
         *abort_s = 0;
         fence_mbar_init();
@@ -194,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (IS_KEY && ok && !*abort_s && my_tiles > 0) projection(my_tiles - 1);
         }
-    } else {
+    } else if (warp < kNormWarp0) {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - kEpiWarp0;   // 0..7
         const int wg = ew >> 2;            // which half of the tiles / TMEM
@@ -202,43 +253,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = 32 * q + lane;     // vector within the tile
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)wg * 256;
         constexpr int wpv = BETA * CHUNKS;
+        constexpr int K = 1 << BETA;
+        float bnd_r[16], cen_r[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            bnd_r[k] = bnd_s[k];
+            cen_r[k] = cen_s[k];
+        }
         for (int i = wg; i < my_tiles; i += 2) {
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
             const int64_t v = tile * kTileRows + row;
             const bool valid = v < n;
+            if (!mbar_wait(&bars[kNormReady + wg], (i >> 1) & 1, abort_s)) break;
             if (!mbar_wait(&bars[kRotFull + wg], (i >> 1) & 1, abort_s)) break;
             tc_fence_after();
-            uint32_t r[32];
-            float ss = 0.f;
-#pragma unroll
-            for (int c = 0; c < CHUNKS; ++c) {
-                tmem_ld32(tl + 32 * c, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int l = 0; l < 32; ++l) ss = fmaf(__uint_as_float(r[l]), __uint_as_float(r[l]), ss);
-            }
-            const float nacc = sqrtf(ss);
-            const float inv = nacc > 0.f ? 1.0f / nacc : 0.f;
+            const float nx = sqrtf(norm_s[wg * kTileRows + row]);
+            // the accumulator holds 2^8 R x; y = R x / ||x||
+            const float inv = nx > 0.f ? (1.0f / (float)(1 << kRScaleLog2)) / nx : 0.f;
             uint32_t words[BETA * CHUNKS];
             float ee = 0.f;
+            uint32_t r[2][32];
+            tmem_ld32(tl, r[0]);
+            tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < CHUNKS; ++c) {
-                tmem_ld32(tl + 32 * c, r);
-                tmem_ld_wait();
+                if (c + 1 < CHUNKS) tmem_ld32(tl + 32 * (c + 1), r[(c + 1) & 1]);
                 uint32_t wp[4] = {0u, 0u, 0u, 0u};
                 uint32_t hp[16], lp[16];
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
-                    const float y = __uint_as_float(r[l]) * inv;
-                    int idx = 0;
+                    const float y = __uint_as_float(r[c & 1][l]) * inv;
+                    const uint32_t idx = bucket_tree<BETA>(y, bnd_r);
 #pragma unroll
-                    for (int p = BETA - 1; p >= 0; --p) {
-                        const bool t = y > bnd_s[idx + (1 << p) - 1];
-                        idx += t ? (1 << p) : 0;
-                        wp[p] |= (uint32_t)t << l;
-                    }
+                    for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
                     if (IS_KEY) {
-                        const float e = y - cen_s[idx];
+                        const float e = y - mux<K>(cen_r, idx);
                         ee = fmaf(e, e, ee);
                         const float es = e * kEScale;
                         const __half h = __float2half_rn(es);
@@ -259,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st16(tl + 32 * c, hp);
                     tmem_st16(tl + 32 * c + 16, lp);
                 }
+                if (c + 1 < CHUNKS) tmem_ld_wait();
             }
             if (IS_KEY) tmem_st_wait();
             tc_fence_before();
@@ -274,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int w2 = 0; w2 < wpv; w2 += 2) *(uint2 *)(dst + w2) = make_uint2(words[w2], words[w2 + 1]);
                 }
-                norm[v] = f32_to_f16_bits(nacc * (1.0f / (float)(1 << kRScaleLog2)));
+                norm[v] = f32_to_f16_bits(nx);
             }
             if (IS_KEY) {
                 if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
@@ -282,16 +332,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const int spk = m >> 5;
                 for (int g = 0; g < spk; ++g) {
-                    tmem_ld32(tl + 128 + 32 * g, r);
+                    tmem_ld32(tl + 128 + 32 * g, r[0]);
                     tmem_ld_wait();
                     uint32_t sw = 0;
 #pragma unroll
-                    for (int l = 0; l < 32; ++l) sw |= (uint32_t)(__uint_as_float(r[l]) >= 0.f) << l;
+                    for (int l = 0; l < 32; ++l) sw |= (uint32_t)(__uint_as_float(r[0][l]) >= 0.f) << l;
                     if (valid) signs[v * spk + g] = sw;
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kTmemEmpty + wg]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ row norms
+        // ||x||^2 of every row of the fp16 input tile, read from the swizzled stage in
+        // shared memory (exact fp16 inputs, fp32 sums); two warps, 64 rows each.
+        const int nw = warp - kNormWarp0;
+        for (int i = 0; i < my_tiles; ++i) {
+            const int slot = i & 1, stage = i % NST;
+            if (i >= 2 && !mbar_wait(&bars[kTmemEmpty + slot], ((i >> 1) - 1) & 1, abort_s)) break;
+            if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) break;
+            const uint8_t *xs = sm + L.X + stage * XSTAGE;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = nw * 64 + h * 32 + lane;
+                float ss = 0.f;
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    const int kb = c >> 3, cc = c & 7;
+                    const uint4 w = *(const uint4 *)(xs + kb * (kTileRows * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+                    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __half22float2(*(const __half2 *)&u[e]);
+                        ss = fmaf(f.x, f.x, ss);
+                        ss = fmaf(f.y, f.y, ss);
+                    }
+                }
+                norm_s[slot * kTileRows + r] = ss;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[kNormReady + slot]);
+                mbar_arrive(&bars[kEmpty + stage]);
             }
         }
     }
