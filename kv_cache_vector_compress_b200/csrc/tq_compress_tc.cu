@@ -28,7 +28,7 @@ constexpr int kTileRows = 128;
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kEpiWarp0 = 2;   // warps 2..9: epilogue (two groups of four)
 constexpr int kNormWarp0 = 10; // warps 10..11: row norms of the input tiles
-constexpr float kEScale = 1024.f;  // residual scale before the fp16 hi/lo split
+constexpr int kCScaleLog2 = 10;  // centroid scale before the fp16 hi/lo split
 
 struct TcSmem {
     // offsets from the 1024-aligned dynamic shared memory base
@@ -41,7 +41,7 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int m, bool is_key) {
     TcSmem L;
     uint32_t o = 0;
     L.R = o;
-    o += 2u * D * D * 2;
+    o += 2u * (is_key ? D + m : D) * D * 2;  // [R; S] (keys) or R (values), hi | lo
     L.S = o;
     if (is_key) o += 2u * m * D * 2;
     L.X = o;
@@ -94,6 +94,17 @@ __device__ __forceinline__ uint32_t bucket_tree(float y, const float (&b)[16]) {
                              : (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]));
         const bool t0 = y > thr;
         return (t3 ? 8u : 0u) | (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ uint32_t umux(const uint32_t *v, uint32_t idx) {
+    if constexpr (N == 1) {
+        return v[0];
+    } else {
+        const uint32_t lo = umux<N / 2>(v, idx);
+        const uint32_t hi = umux<N / 2>(v + N / 2, idx);
+        return (idx & (N / 2)) ? hi : lo;
     }
 }
 
@@ -169,10 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmap);
-            const uint32_t rbytes = 2u * D * D * 2;
+            const uint32_t rbytes = 2u * (IS_KEY ? D + m : D) * D * 2;
             const uint32_t sbytes = IS_KEY ? 2u * m * D * 2 : 0u;
             mbar_arrive_expect_tx(&bars[kOpnd], rbytes + sbytes);
-            bulk_load(sm + L.R, P.Rsw, rbytes, &bars[kOpnd]);
+            bulk_load(sm + L.R, IS_KEY ? P.RSsw : P.Rsw, rbytes, &bars[kOpnd]);
             if (IS_KEY) bulk_load(sm + L.S, P.Ssw, sbytes, &bars[kOpnd]);
             int issued = 0;
             for (int i = 0; i < my_tiles; ++i) {
@@ -196,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_rot = idesc_f16_f32(128, D);
+            const int rowsB = IS_KEY ? D + m : D;
+            const uint32_t idesc_rot = idesc_f16_f32(128, rowsB);
             const uint32_t idesc_prj = idesc_f16_f32(128, m > 0 ? m : 16);
             const uint32_t sR = smem_u32(sm + L.R), sS = smem_u32(sm + L.S), sX = smem_u32(sm + L.X);
             bool ok = mbar_wait(&bars[kOpnd], 0, abort_s);
@@ -204,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int slot = j & 1;
                 if (!mbar_wait(&bars[kEReady + slot], (j >> 1) & 1, abort_s)) return false;
                 tc_fence_after();
-                const uint32_t acc = tmem + slot * 256 + 128;
+                const uint32_t acc = tmem + slot * 256 + D + m;
                 const uint32_t sbytes = (uint32_t)m * D * 2;
                 uint32_t first = 0;
 #pragma unroll 1
@@ -222,10 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&bars[kProjFull + slot]);
                 return true;
             };
-            for (int i = 0; ok && i < my_tiles; ++i) {
+            auto rotation = [&](int i) -> bool {
                 const int slot = i & 1, stage = i % NST;
-                if (i >= 2 && !mbar_wait(&bars[kTmemEmpty + slot], ((i >> 1) - 1) & 1, abort_s)) break;
-                if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) break;
+                if (i >= 2 && !mbar_wait(&bars[kTmemEmpty + slot], ((i >> 1) - 1) & 1, abort_s)) return false;
+                if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) return false;
                 tc_fence_after();
                 const uint32_t acc = tmem + slot * 256;
                 const uint32_t xbase = sX + stage * XSTAGE;
@@ -235,15 +247,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int k = 0; k < KSTEPS; ++k) {
                         const uint32_t aoff = (uint32_t)(k >> 2) * (kTileRows * 128) + (k & 3) * 32;
-                        const uint32_t boff = (uint32_t)pass * (D * D * 2) + (uint32_t)(k >> 2) * (D * 128) + (k & 3) * 32;
+                        const uint32_t boff = (uint32_t)pass * (rowsB * D * 2) + (uint32_t)(k >> 2) * (rowsB * 128) +
+                                              (k & 3) * 32;
                         mma_ss(acc, sdesc_sw128(xbase + aoff), sdesc_sw128(sR + boff), idesc_rot, first);
                         first = 1;
                     }
                 mma_commit(&bars[kEmpty + stage]);
                 mma_commit(&bars[kRotFull + slot]);
-                if (IS_KEY && i >= 1 && !projection(i - 1)) break;
+                return true;
+            };
+            // Two tiles in flight (one per TMEM slot); the projection of tile j goes out as soon
+            // as its residual is ready, before the rotation that reuses tile j's slot.
+            if (ok && my_tiles > 0) ok = rotation(0);
+            if (ok && my_tiles > 1) ok = rotation(1);
+            for (int j = 0; ok && j < my_tiles; ++j) {
+                if (IS_KEY && !projection(j)) break;
+                if (j + 2 < my_tiles && !rotation(j + 2)) break;
             }
-            if (IS_KEY && ok && !*abort_s && my_tiles > 0) projection(my_tiles - 1);
         }
     } else if (warp < kNormWarp0) {
         // ------------------------------------------------------------ epilogue
@@ -255,10 +275,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int wpv = BETA * CHUNKS;
         constexpr int K = 1 << BETA;
         float bnd_r[16], cen_r[16];
+        uint32_t cbit_r[16];  // (hi << 16) | lo: fp16 split of centroid * 2^kCScaleLog2
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             bnd_r[k] = bnd_s[k];
             cen_r[k] = cen_s[k];
+            const float cs = cen_r[k] * (float)(1 << kCScaleLog2);
+            const __half h = __float2half_rn(cs);
+            const __half lo = __float2half_rn(cs - __half2float(h));
+            cbit_r[k] = ((uint32_t)__half_as_ushort(h) << 16) | (uint32_t)__half_as_ushort(lo);
         }
         for (int i = wg; i < my_tiles; i += 2) {
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
@@ -289,16 +314,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (IS_KEY) {
                         const float e = y - mux<K>(cen_r, idx);
                         ee = fmaf(e, e, ee);
-                        const float es = e * kEScale;
-                        const __half h = __float2half_rn(es);
-                        const __half lo = __float2half_rn(es - __half2float(h));
-                        const uint32_t hb = __half_as_ushort(h), lb = __half_as_ushort(lo);
+                        const uint32_t cb = umux<K>(cbit_r, idx);
                         if (l & 1) {
-                            hp[l >> 1] |= hb << 16;
-                            lp[l >> 1] |= lb << 16;
+                            hp[l >> 1] = __byte_perm(hp[l >> 1], cb, 0x7632);
+                            lp[l >> 1] = __byte_perm(lp[l >> 1], cb, 0x5410);
                         } else {
-                            hp[l >> 1] = hb;
-                            lp[l >> 1] = lb;
+                            hp[l >> 1] = cb;
+                            lp[l >> 1] = cb;
                         }
                     }
                 }
@@ -330,13 +352,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
                 if (!mbar_wait(&bars[kProjFull + wg], (i >> 1) & 1, abort_s)) break;
                 tc_fence_after();
+                // p = S u - S' c[idx]: S u from the rotation accumulator (2^8 S x), S' c from the
+                // projection accumulator (2^(kCScaleLog2 + kSScaleLog2) S' c)
                 const int spk = m >> 5;
+                const float pun = 1.0f / (float)(1 << (kCScaleLog2 + kSScaleLog2));
                 for (int g = 0; g < spk; ++g) {
-                    tmem_ld32(tl + 128 + 32 * g, r[0]);
+                    tmem_ld32(tl + D + 32 * g, r[0]);
+                    tmem_ld32(tl + D + m + 32 * g, r[1]);
                     tmem_ld_wait();
                     uint32_t sw = 0;
 #pragma unroll
-                    for (int l = 0; l < 32; ++l) sw |= (uint32_t)(__uint_as_float(r[0][l]) >= 0.f) << l;
+                    for (int l = 0; l < 32; ++l) {
+                        const float pv = fmaf(__uint_as_float(r[0][l]), inv, -__uint_as_float(r[1][l]) * pun);
+                        sw |= (uint32_t)(pv >= 0.f) << l;
+                    }
                     if (valid) signs[v * spk + g] = sw;
                 }
                 tc_fence_before();
@@ -435,7 +464,8 @@ cudaError_t launch_tc(const Prepared &P, const void *x, int64_t n, uint32_t *cod
 bool compress_tc_supported(const Prepared &P, bool is_key, bool x_f16) {
     if (!x_f16) return false;
     if (P.d != 128 && P.d != 64) return false;
-    if (is_key && (P.m < 32 || P.m > 128 || P.m % 32)) return false;
+    // keys keep [R x | S x] and the projection in one 256-column TMEM slot
+    if (is_key && (P.m < 32 || P.m % 32 || P.d + 2 * P.m > 256)) return false;
     return true;
 }
 

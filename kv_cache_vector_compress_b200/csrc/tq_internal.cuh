@@ -34,6 +34,7 @@ struct WsLayout {
     size_t SpT;        // fp32 [d, m]      (S R^T) transposed
     size_t Rsw;        // fp16 hi | lo of R * 2^kRScaleLog2, tensor-core operand layout
     size_t Ssw;        // fp16 hi | lo of (S R^T) * 2^kSScaleLog2, same layout
+    size_t RSsw;       // fp16 hi | lo of [R; S] * 2^kRScaleLog2 (d + m rows), same layout
     size_t total;
 };
 
@@ -78,6 +79,8 @@ inline WsLayout ws_layout(int d, int m) {
     o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * d, 1024);
     L.Ssw = o;
     o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * (m > 0 ? m : 1), 1024);
+    L.RSsw = o;
+    o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * (d + m), 1024);
     L.total = o;
     return L;
 }
@@ -87,7 +90,7 @@ struct Prepared {
     int d, m, kbeta, vbeta;
     const Codebooks *cb;
     const float *R, *RT, *ST, *SpT;
-    const uint16_t *Rsw, *Ssw;
+    const uint16_t *Rsw, *Ssw, *RSsw;
 };
 
 inline Prepared prepared_view(const tq_params *p) {
@@ -105,6 +108,7 @@ inline Prepared prepared_view(const tq_params *p) {
     v.SpT = (const float *)(w + L.SpT);
     v.Rsw = (const uint16_t *)(w + L.Rsw);
     v.Ssw = (const uint16_t *)(w + L.Ssw);
+    v.RSsw = (const uint16_t *)(w + L.RSsw);
     return v;
 }
 

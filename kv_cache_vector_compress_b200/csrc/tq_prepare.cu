@@ -32,6 +32,22 @@ __global__ void prepare_kernel(const float *__restrict__ R, const float *__restr
         Rhi[off] = __half_as_ushort(hi);
         Rlo[off] = __half_as_ushort(lo);
     }
+    // keys' rotation operand [R; S] * 2^s split into fp16 hi + lo, d + m rows
+    {
+        const int rows = d + (m > 0 ? m : 0);
+        uint16_t *Xhi = (uint16_t *)(ws + L.RSsw);
+        uint16_t *Xlo = Xhi + (size_t)d * rows;
+        for (int64_t e = tid; e < (int64_t)rows * d; e += nth) {
+            const int i = (int)(e / d), j = (int)(e % d);
+            const float v = (i < d) ? R[(int64_t)i * d + j] : S[(int64_t)(i - d) * d + j];
+            const float sv = v * (float)(1 << kRScaleLog2);
+            const __half hi = __float2half_rn(sv);
+            const __half lo = __float2half_rn(sv - __half2float(hi));
+            const size_t off = sw128_offset(rows, i, j) / 2;
+            Xhi[off] = __half_as_ushort(hi);
+            Xlo[off] = __half_as_ushort(lo);
+        }
+    }
     if (m <= 0) return;
     for (int64_t e = tid; e < (int64_t)m * d; e += nth) {
         int a = (int)(e / d), j = (int)(e % d);

@@ -31,23 +31,36 @@ inline int rows_per_pass(int d, int m, int cap_regs) {
 
 // ------------------------------------------------------------------ query prep
 
+constexpr int kQprepRows = 8;
+
+// q_rot = R q and sq = S q for kQprepRows query rows per block: each thread owns one output
+// coordinate and carries one accumulator per row (the R^T / S^T row it reads is shared).
 __global__ void qprep_kernel(Prepared P, const float *__restrict__ q, int64_t rows,
                              float *__restrict__ out) {
-    extern __shared__ float qs[];
+    extern __shared__ float qs[];  // [kQprepRows][d]
     const int d = P.d, m = P.m;
-    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
-        for (int j = threadIdx.x; j < d; j += blockDim.x) qs[j] = q[row * d + j];
-        __syncthreads();
-        float *o = out + row * (d + m);
-        for (int i = threadIdx.x; i < d; i += blockDim.x) {
-            float acc = 0.f;
-            for (int j = 0; j < d; ++j) acc = fmaf(P.RT[(int64_t)j * d + i], qs[j], acc);
-            o[i] = acc;
+    for (int64_t r0 = (int64_t)blockIdx.x * kQprepRows; r0 < rows; r0 += (int64_t)gridDim.x * kQprepRows) {
+        const int nr = (int)min((int64_t)kQprepRows, rows - r0);
+        for (int e = threadIdx.x; e < kQprepRows * d; e += blockDim.x) {
+            const int r = e / d, j = e % d;
+            qs[e] = r < nr ? q[(r0 + r) * d + j] : 0.f;
         }
-        for (int a = threadIdx.x; a < m; a += blockDim.x) {
-            float acc = 0.f;
-            for (int j = 0; j < d; ++j) acc = fmaf(P.ST[(int64_t)j * m + a], qs[j], acc);
-            o[d + a] = acc;
+        __syncthreads();
+        for (int i = threadIdx.x; i < d + m; i += blockDim.x) {
+            const bool rot = i < d;
+            const float *mat = rot ? P.RT + i : P.ST + (i - d);
+            const int ld = rot ? d : m;
+            float acc[kQprepRows];
+#pragma unroll
+            for (int r = 0; r < kQprepRows; ++r) acc[r] = 0.f;
+            for (int j = 0; j < d; ++j) {
+                const float w = mat[(int64_t)j * ld];
+#pragma unroll
+                for (int r = 0; r < kQprepRows; ++r) acc[r] = fmaf(w, qs[r * d + j], acc[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < kQprepRows; ++r)
+                if (r < nr) out[(r0 + r) * (d + m) + i] = acc[r];
         }
         __syncthreads();
     }
@@ -397,8 +410,11 @@ size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk) {
 
 cudaError_t launch_qprep(const Prepared &P, const ScoreProblem &sp, float *qprep, cudaStream_t s) {
     const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
-    int blocks = (int)(rows < 148 * 8 ? rows : 148 * 8);
-    qprep_kernel<<<blocks, 128, sizeof(float) * P.d, s>>>(P, sp.q, rows, qprep);
+    const int64_t groups = (rows + kQprepRows - 1) / kQprepRows;
+    int blocks = (int)(groups < 148 * 8 ? groups : 148 * 8);
+    const size_t smem = sizeof(float) * kQprepRows * P.d;
+    cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    qprep_kernel<<<blocks, 128, smem, s>>>(P, sp.q, rows, qprep);
     return cudaGetLastError();
 }
 
