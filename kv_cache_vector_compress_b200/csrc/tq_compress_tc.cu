@@ -295,19 +295,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float nx = sqrtf(norm_s[wg * kTileRows + row]);
             // the accumulator holds 2^8 R x; y = R x / ||x||
             const float inv = nx > 0.f ? (1.0f / (float)(1 << kRScaleLog2)) / nx : 0.f;
-            uint32_t words[BETA * CHUNKS];
             float ee = 0.f;
-            uint32_t r[2][32];
-            tmem_ld32(tl, r[0]);
-            tmem_ld_wait();
-#pragma unroll
+            uint32_t r[32];
+            uint32_t *dst = codes + v * wpv;
+            // chunks of 32 coordinates; the loop stays rolled so the unrolled body fits the
+            // instruction cache, and each chunk's code words go straight to global memory
+#pragma unroll 1
             for (int c = 0; c < CHUNKS; ++c) {
-                if (c + 1 < CHUNKS) tmem_ld32(tl + 32 * (c + 1), r[(c + 1) & 1]);
+                tmem_ld32(tl + 32 * c, r);
+                tmem_ld_wait();
                 uint32_t wp[4] = {0u, 0u, 0u, 0u};
                 uint32_t hp[16], lp[16];
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
-                    const float y = __uint_as_float(r[c & 1][l]) * inv;
+                    const float y = __uint_as_float(r[l]) * inv;
                     const uint32_t idx = bucket_tree<BETA>(y, bnd_r);
 #pragma unroll
                     for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
@@ -324,30 +325,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-#pragma unroll
-                for (int p = 0; p < BETA; ++p) words[c * BETA + p] = wp[p];
                 if (IS_KEY) {
                     tmem_st16(tl + 32 * c, hp);
                     tmem_st16(tl + 32 * c + 16, lp);
                 }
-                if (c + 1 < CHUNKS) tmem_ld_wait();
+                if (valid) {
+#pragma unroll
+                    for (int p = 0; p < BETA; ++p) dst[c * BETA + p] = wp[p];
+                }
             }
             if (IS_KEY) tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(IS_KEY ? &bars[kEReady + wg] : &bars[kTmemEmpty + wg]);
-            if (valid) {
-                uint32_t *dst = codes + v * wpv;
-                if constexpr ((wpv & 3) == 0) {
-#pragma unroll
-                    for (int w4 = 0; w4 < wpv; w4 += 4)
-                        *(uint4 *)(dst + w4) = make_uint4(words[w4], words[w4 + 1], words[w4 + 2], words[w4 + 3]);
-                } else {
-#pragma unroll
-                    for (int w2 = 0; w2 < wpv; w2 += 2) *(uint2 *)(dst + w2) = make_uint2(words[w2], words[w2 + 1]);
-                }
-                norm[v] = f32_to_f16_bits(nx);
-            }
+            if (valid) norm[v] = f32_to_f16_bits(nx);
             if (IS_KEY) {
                 if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
                 if (!mbar_wait(&bars[kProjFull + wg], (i >> 1) & 1, abort_s)) break;
@@ -356,14 +347,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // projection accumulator (2^(kCScaleLog2 + kSScaleLog2) S' c)
                 const int spk = m >> 5;
                 const float pun = 1.0f / (float)(1 << (kCScaleLog2 + kSScaleLog2));
+#pragma unroll 1
                 for (int g = 0; g < spk; ++g) {
-                    tmem_ld32(tl + D + 32 * g, r[0]);
-                    tmem_ld32(tl + D + m + 32 * g, r[1]);
+                    uint32_t r2[32];
+                    tmem_ld32(tl + D + 32 * g, r);
+                    tmem_ld32(tl + D + m + 32 * g, r2);
                     tmem_ld_wait();
                     uint32_t sw = 0;
 #pragma unroll
                     for (int l = 0; l < 32; ++l) {
-                        const float pv = fmaf(__uint_as_float(r[0][l]), inv, -__uint_as_float(r[1][l]) * pun);
+                        const float pv = fmaf(__uint_as_float(r[l]), inv, -__uint_as_float(r2[l]) * pun);
                         sw |= (uint32_t)(pv >= 0.f) << l;
                     }
                     if (valid) signs[v * spk + g] = sw;
