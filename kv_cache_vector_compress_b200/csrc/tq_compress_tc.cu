@@ -71,29 +71,24 @@ enum BarIdx {
 };
 
 // Code of y against ascending boundaries b[0..2^BETA-2] (#{k : b[k] < y}) by a binary
-// search whose thresholds are selected from registers.
+// search whose thresholds are selected from registers; t[p] receives bit p of the code.
 template <int BETA>
-__device__ __forceinline__ uint32_t bucket_tree(float y, const float (&b)[16]) {
+__device__ __forceinline__ void bucket_bits(float y, const float (&b)[16], bool (&t)[4]) {
     if constexpr (BETA == 1) {
-        return y > b[0] ? 1u : 0u;
+        t[0] = y > b[0];
     } else if constexpr (BETA == 2) {
-        const bool t1 = y > b[1];
-        const bool t0 = y > (t1 ? b[2] : b[0]);
-        return (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+        t[1] = y > b[1];
+        t[0] = y > (t[1] ? b[2] : b[0]);
     } else if constexpr (BETA == 3) {
-        const bool t2 = y > b[3];
-        const bool t1 = y > (t2 ? b[5] : b[1]);
-        const float thr = t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]);
-        const bool t0 = y > thr;
-        return (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+        t[2] = y > b[3];
+        t[1] = y > (t[2] ? b[5] : b[1]);
+        t[0] = y > (t[2] ? (t[1] ? b[6] : b[4]) : (t[1] ? b[2] : b[0]));
     } else {
-        const bool t3 = y > b[7];
-        const bool t2 = y > (t3 ? b[11] : b[3]);
-        const bool t1 = y > (t3 ? (t2 ? b[13] : b[9]) : (t2 ? b[5] : b[1]));
-        const float thr = t3 ? (t2 ? (t1 ? b[14] : b[12]) : (t1 ? b[10] : b[8]))
-                             : (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]));
-        const bool t0 = y > thr;
-        return (t3 ? 8u : 0u) | (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+        t[3] = y > b[7];
+        t[2] = y > (t[3] ? b[11] : b[3]);
+        t[1] = y > (t[3] ? (t[2] ? b[13] : b[9]) : (t[2] ? b[5] : b[1]));
+        t[0] = y > (t[3] ? (t[2] ? (t[1] ? b[14] : b[12]) : (t[1] ? b[10] : b[8]))
+                         : (t[2] ? (t[1] ? b[6] : b[4]) : (t[1] ? b[2] : b[0])));
     }
 }
 
@@ -130,7 +125,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int CHUNKS = D / 32;
     constexpr uint32_t XSTAGE = kTileRows * D * 2;
     const int m = IS_KEY ? P.m : 0;
-    constexpr int beta = BETA;
     const TcSmem L = tc_smem_layout(D, m, IS_KEY);
     const int NST = L.nst;
 
@@ -142,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *tmem_s = (uint32_t *)(cen_s + kMaxLevels);
     volatile int *abort_s = (volatile int *)(tmem_s + 1);
     float *norm_s = (float *)(sm + L.misc + 256);  // [2 slots][128 rows] squared norms
+    uint32_t *cbit_s = (uint32_t *)(sm + L.misc + 256 + 1024);  // centroid fp16 hi/lo bits
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
@@ -165,7 +160,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (threadIdx.x < kMaxLevels) {
         bnd_s[threadIdx.x] = IS_KEY ? P.cb->kb[threadIdx.x] : P.cb->vb[threadIdx.x];
-        cen_s[threadIdx.x] = IS_KEY ? P.cb->kc[threadIdx.x] : P.cb->vc[threadIdx.x];
+        const float c = IS_KEY ? P.cb->kc[threadIdx.x] : P.cb->vc[threadIdx.x];
+        cen_s[threadIdx.x] = c;
+        const float cs = c * (float)(1 << kCScaleLog2);
+        const __half h = __float2half_rn(cs);
+        const __half lo = __float2half_rn(cs - __half2float(h));
+        cbit_s[threadIdx.x] = ((uint32_t)__half_as_ushort(h) << 16) | (uint32_t)__half_as_ushort(lo);
     }
     if (warp == 0) {
         tmem_alloc(tmem_s, 512);
@@ -273,18 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = 32 * q + lane;     // vector within the tile
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)wg * 256;
         constexpr int wpv = BETA * CHUNKS;
-        constexpr int K = 1 << BETA;
-        float bnd_r[16], cen_r[16];
-        uint32_t cbit_r[16];  // (hi << 16) | lo: fp16 split of centroid * 2^kCScaleLog2
+        float bnd_r[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            bnd_r[k] = bnd_s[k];
-            cen_r[k] = cen_s[k];
-            const float cs = cen_r[k] * (float)(1 << kCScaleLog2);
-            const __half h = __float2half_rn(cs);
-            const __half lo = __float2half_rn(cs - __half2float(h));
-            cbit_r[k] = ((uint32_t)__half_as_ushort(h) << 16) | (uint32_t)__half_as_ushort(lo);
-        }
+        for (int k = 0; k < 16; ++k) bnd_r[k] = bnd_s[k];
         for (int i = wg; i < my_tiles; i += 2) {
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
             const int64_t v = tile * kTileRows + row;
@@ -309,13 +300,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
                     const float y = __uint_as_float(r[l]) * inv;
-                    const uint32_t idx = bucket_tree<BETA>(y, bnd_r);
+                    bool t[4];
+                    bucket_bits<BETA>(y, bnd_r, t);
+                    uint32_t idx = 0;
 #pragma unroll
-                    for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
+                    for (int p = 0; p < BETA; ++p) {
+                        if (t[p]) wp[p] |= 1u << l;
+                        idx |= (t[p] ? 1u : 0u) << p;
+                    }
                     if (IS_KEY) {
-                        const float e = y - mux<K>(cen_r, idx);
+                        // centroid and its fp16 hi/lo bit pattern from shared-memory tables
+                        const float e = y - cen_s[idx];
                         ee = fmaf(e, e, ee);
-                        const uint32_t cb = umux<K>(cbit_r, idx);
+                        const uint32_t cb = cbit_s[idx];
                         if (l & 1) {
                             hp[l >> 1] = __byte_perm(hp[l >> 1], cb, 0x7632);
                             lp[l >> 1] = __byte_perm(lp[l >> 1], cb, 0x5410);
