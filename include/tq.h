@@ -21,8 +21,9 @@
  * Conventions (all functions):
  *   - Every call returns a tq_status.  Argument errors are detected on the host and
  *     returned before anything is launched; nothing is written in that case.
- *   - The caller allocates and owns every buffer.  The library never allocates,
- *     frees or keeps device memory and holds no global mutable state.
+ *   - The caller allocates and owns every buffer.  The library never allocates or
+ *     frees device memory; the one device memory it keeps is the fixed scratch array
+ *     of tq_attend_static (declared last), which exists only for that call.
  *   - Device work is enqueued asynchronously on the caller's stream; results are
  *     ready when that stream is synchronised.  Outputs are bit-identical run to run.
  *   - Device pointers must be 16-byte aligned (TQ_ERR_INVALID_ARG otherwise).
@@ -179,6 +180,29 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
                     const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm,
                     float scale, float *out, void *scratch, size_t scratch_bytes,
                     int32_t *dev_status, tq_stream_t stream);
+
+/*
+ * tq_attend_static -- tq_attend for callers that cannot allocate device memory when they call.
+ * (The pages have no counterpart: this is an addition of the library.)
+ * A serving loop whose device memory is all handed to its own pool up front, or code that must
+ * not pay the device synchronisation cudaMalloc / cudaFree can cause inside a decode step, has
+ * no scratch buffer to pass.  This call takes its scratch from a library-owned device array of
+ * TQ_STATIC_SCRATCH_BYTES instead; every GPU that loads the library holds that array until the
+ * process exits.  Arguments and results are those of tq_attend, without scratch/scratch_bytes.
+ *   - Problems whose tq_attend_scratch_bytes(...) exceeds TQ_STATIC_SCRATCH_BYTES are rejected
+ *     with TQ_ERR_UNSUPPORTED before any work; use tq_attend with your own scratch for them.
+ *   - The call never allocates: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's address on that device (with that device
+ *     current); make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents (nothing in it needs
+ *     to start at zero).  Calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on it: serialise them.
+ */
+#define TQ_STATIC_SCRATCH_BYTES (16u << 20)
+tq_status tq_attend_static(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                           const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                           const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm,
+                           float scale, float *out, int32_t *dev_status, tq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -62,9 +62,15 @@ _lib.tq_attend.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P
                            _SZ, _P, _P]
 _lib.tq_attend.restype = _I
 
+_lib.tq_attend_static.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P,
+                                  _P, _P]
+_lib.tq_attend_static.restype = _I
+
+TQ_STATIC_SCRATCH_BYTES = 16 << 20
+
 EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_workspace_bytes", "tq_prepare",
            "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores",
-           "tq_attend_scratch_bytes", "tq_attend"]
+           "tq_attend_scratch_bytes", "tq_attend", "tq_attend_static"]
 
 
 class TQError(RuntimeError):
@@ -223,4 +229,19 @@ def tq_attend(p: Params, q: torch.Tensor, keys, values, Hkv: int, T: int, scale:
     _check(_lib.tq_attend(p.ref, _ptr(q), B, Hq, Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr),
                           _ptr(vc), _ptr(vn), float(scale), _ptr(out), _ptr(scratch), scratch.numel(),
                           _ptr(dev_status), _stream()), "tq_attend")
+    return out
+
+
+def tq_attend_static(p: Params, q: torch.Tensor, keys, values, Hkv: int, T: int, scale: float = 0.0, out=None,
+                     dev_status=None):
+    """tq_attend with the library-owned scratch array (no scratch argument, no allocation inside
+    the library).  `out` may be passed in so that the call allocates nothing at all."""
+    B, Hq, Nq, d = q.shape
+    kc, ks, kn, kr = keys
+    vc, vn = values
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.float32, device=q.device)
+    _check(_lib.tq_attend_static(p.ref, _ptr(q), B, Hq, Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr),
+                                 _ptr(vc), _ptr(vn), float(scale), _ptr(out), _ptr(dev_status), _stream()),
+           "tq_attend_static")
     return out
