@@ -183,18 +183,36 @@ def run_reference(args):
 
 # -------------------------------------------------------------------- GPU arm
 
+def traffic_per_unit(kernel: str):
+    """DRAM bytes per unit of `kernel` from the committed ncu summary, or None when the kernel's
+    source has changed since the counters were taken (the summary records its sha1)."""
+    import hashlib
+    try:
+        lines = open(os.path.join(ROOT, "profiles", "dram_traffic.md")).read().splitlines()
+    except OSError:
+        return None
+    for ln in lines:
+        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == kernel:
+            src, sha, per_unit = cells[1], cells[2], cells[3]
+            try:
+                cur = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:12]
+                if cur == sha:
+                    return float(per_unit)
+            except (OSError, ValueError):
+                return None
+    return None
+
+
 def run_tq(args):
     import numpy as np
     import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from kv_cache_vector_compress_b200 import dist as tqdist
+    ri = tqdist.rank_info()
+    world, rank, local = ri.world, ri.rank, ri.local
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    tqdist.init("nccl", timeout_s=120)
     from kv_cache_vector_compress_b200 import synth, tq
 
     w = dict(W3)
@@ -204,7 +222,7 @@ def run_tq(args):
     B, Hq, Hkv, Nq, T = w["B"], w["Hq"], w["Hkv"], w["Nq"], w["T"]
     n = B * Hkv * T
     s = synth.seeds(3)
-    off = 7919 * rank
+    off = tqdist.seed_offset(rank)
     R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
     S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
     p = tq.Params(d, bits, m, R, S)
@@ -236,8 +254,7 @@ def run_tq(args):
             ev[3].record(stream)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        tqdist.barrier()
         torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -260,10 +277,7 @@ def run_tq(args):
         op_ms["compress_keys"] += e[0].elapsed_time(e[1]) / args.steps
         op_ms["compress_values"] += e[1].elapsed_time(e[2]) / args.steps
         op_ms["attend"] += e[2].elapsed_time(e[3]) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = tqdist.max_over_ranks(ms, device="cuda")
     ms_step = ms / args.steps
 
     # end to end through the public API: pinned host K/V in, attention output out
@@ -293,10 +307,7 @@ def run_tq(args):
     a1.record(stream)
     barrier()
     e2e_ms = a0.elapsed_time(a1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = tqdist.max_over_ranks(e2e_ms, device="cuda")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -314,13 +325,9 @@ def run_tq(args):
         breakdown["attend"]["packed_keys_scored_per_s"] = n / (op_ms["attend"] * 1e-3)
         dom = max(op_ms, key=lambda k: op_ms[k])
         ach = ab[dom] / (op_ms[dom] * 1e-3) / 1e9
-        traffic = None
-        try:
-            with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-                traffic = json.load(f).get(dom)
-        except Exception:
-            traffic = None
-        value = world * n / (ms_step * 1e-3)
+        tpu = traffic_per_unit(dom)
+        traffic = None if tpu is None else tpu * n
+        value = tqdist.weak_scaling_value(n, world, ms_step * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -339,9 +346,8 @@ def run_tq(args):
         if cpu:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    tqdist.barrier()
+    tqdist.destroy()
     return 0
 
 

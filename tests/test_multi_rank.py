@@ -1,0 +1,79 @@
+"""The N > 1 path's host logic on CPU: two gloo ranks, each compressing and attending its own
+(batch, KV-head) slice with the oracle as the stand-in compute, then the max-over-ranks timing
+reduction and the whole-job throughput the benchmark reports."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+from kv_cache_vector_compress_b200 import dist as tqdist
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import time
+
+    import oracle
+    from kv_cache_vector_compress_b200 import synth
+    ri = tqdist.init("gloo", timeout_s=60)
+    assert (ri.rank, ri.world) == (rank, world)
+    d, m, bits, T, G = 64, 32, 3, 256, 2
+    off = tqdist.seed_offset(rank)
+    R = synth.rotation(d, 1)
+    S = synth.gaussian(m, d, 2)
+    K = synth.gaussian(T, d, 3 + off).astype(np.float16)
+    V = synth.gaussian(T, d, 4 + off).astype(np.float16)
+    q = synth.gaussian(G, d, 5 + off).reshape(1, G, 1, d)
+    tqdist.barrier()
+    t0 = time.perf_counter()
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    v = oracle.compress(V, R, None, bits, is_key=False)
+    o = oracle.attend(q, R, S, bits, 1, G, 1, 1, T, k["codes"], k["signs"], k["norm"], k["rnorm"],
+                      v["codes"], v["norm"])
+    elapsed = time.perf_counter() - t0 + 0.05 * rank  # make the ranks' times differ
+    tqdist.barrier()
+    mx = tqdist.max_over_ranks(elapsed)
+    out_q.put((rank, elapsed, mx, float(np.abs(o).sum()), tqdist.weak_scaling_value(T, world, mx)))
+    tqdist.destroy()
+
+
+def test_two_gloo_ranks_time_as_max_and_work_independently():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort()
+    times = [r[1] for r in res]
+    for r in res:
+        assert r[2] == pytest.approx(max(times))            # every rank sees the max
+        assert r[4] == pytest.approx(world * 256 / max(times))  # whole-job weak-scaling value
+    assert res[0][3] != res[1][3]  # different seeds: the ranks did their own work
+
+
+@pytest.mark.parametrize("n,world", [(10, 2), (7, 3), (256, 8), (1, 4), (0, 2)])
+def test_shards_cover_every_unit_once(n, world):
+    seen = []
+    for r in range(world):
+        s, c = tqdist.shard(n, world, r)
+        seen.extend(range(s, s + c))
+    assert seen == list(range(n))
+
+
+def test_single_rank_is_identity():
+    assert tqdist.max_over_ranks(3.5) == 3.5
+    assert tqdist.rank_info().world >= 1
