@@ -5,15 +5,21 @@
 // dequantized values; "turboquant-pytorch", nav.superapi.store, 常见使用模式 and 核心 API):
 //   s_tr = ||k_t|| ( <q_rot_r, c[kidx_t]> + rho_t sqrt(pi/2)/m <sq_r, 2 sign_t - 1> )
 //   o_rot_r = sum_t softmax_t(scale s_tr) ||v_t|| c[vidx_t],   out_r = R^T o_rot_r
-// Per warp and 16-token block, three m16n8k16 products (fp16 operands, fp32 accumulate):
+// Per warp and 16-token block, three kinds of m16n8k16 products (fp16 operands, fp32 accumulate):
 //   C1[t, r] = Khat[t, :] . Qrot[r, :]      A = decoded key centroids, B = rotated queries
 //   C2[t, r] = Sgn[t, :]  . SQ[r, :]        A = +-1 sign matrix,        B = S q
 //   O[j, r] += Vhat[j, t] . P[t, r]         A = decoded value centroids, B = probabilities
-// The A fragments come from the planar code words with shifts, masks and a small pair
-// look-up table in shared memory (two fp16 centroids per 32-bit entry); the queries stay in
-// registers.  With SPLIT the centroids and queries are carried as fp16 hi + lo pairs (three
-// products), which keeps the raw scores at fp32-level accuracy; fused attention uses the
-// single product, whose error is far below the output tolerance after the softmax average.
+// A fragments come from the planar code words with shifts, masks and small pair look-up tables
+// in shared memory (two fp16 centroids per 32-bit entry; keys carry centroid hi + lo in one
+// 64-bit entry); the queries stay in registers.  Scores are carried at split precision (centroid
+// hi + lo, query hi + lo): with large key norms a single fp16 product moves the softmax logits by
+// more than the output tolerance allows.  When a KV head has at most four query rows (decode with
+// GQA group <= 4), the queries' hi and lo parts fill the eight MMA columns, so one product per
+// centroid part carries both, and the halves are summed with one shuffle.
+//
+// Each warp streams its own contiguous token range through a two-stage cp.async ring (no block
+// barrier in the main loop); the four warps' softmax states are merged at the end and written as
+// one split-context partial (max, sum, o_rot) per row for attend_combine_kernel.
 #include <math.h>
 
 #include "tq_common.cuh"
@@ -24,7 +30,7 @@ namespace tq {
 namespace {
 
 constexpr int kThreadsMma = 128;
-constexpr int kStageTok = 128;
+constexpr int kWarpStage = 32;  // tokens per warp stage (two 16-token blocks)
 constexpr int kRowsPerCta = 8;
 
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -35,9 +41,10 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src)
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "n"(BYTES)
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -46,83 +53,111 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ uint32_t lut_at(const uint32_t *lut, uint32_t byte_offset) {
+__device__ __forceinline__ uint32_t lut32(const uint32_t *lut, uint32_t byte_offset) {
     return *(const uint32_t *)((const char *)lut + byte_offset);
+}
+__device__ __forceinline__ uint2 lut64(const uint2 *lut, uint32_t byte_offset) {
+    return *(const uint2 *)((const char *)lut + byte_offset);
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
 }
+__device__ __forceinline__ float hi_part(float x) { return __half2float(__float2half_rn(x)); }
 
 // power-of-two scale that brings max|x| into [2^9, 2^10)
 __device__ __forceinline__ int scale_exp(float maxabs) {
     if (!(maxabs > 0.f) || !isfinite(maxabs)) return 0;
     int e;
-    frexpf(maxabs, &e);  // maxabs = f * 2^e, f in [0.5, 1)
+    frexpf(maxabs, &e);
     return 10 - e;
 }
 
+// Copy N consecutive 32-bit words (16-byte aligned when N % 4 == 0) into registers.
+template <int N>
+__device__ __forceinline__ void load_words(const uint32_t *p, uint32_t (&w)[N]) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            const uint4 v = *(const uint4 *)(p + i);
+            w[i] = v.x;
+            w[i + 1] = v.y;
+            w[i + 2] = v.z;
+            w[i + 3] = v.w;
+        }
+    } else if constexpr (N % 2 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 2) {
+            const uint2 v = *(const uint2 *)(p + i);
+            w[i] = v.x;
+            w[i + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) w[i] = p[i];
+    }
+}
+
+// Copy `words` 32-bit words from global to shared memory with the widest cp.async the
+// per-record word count allows (records are 16/8/4-byte multiples and so is every offset).
+template <int RECW>
+__device__ __forceinline__ void stage_copy(uint32_t *dst, const uint32_t *src, int words, int lane) {
+    constexpr int G = (RECW % 4 == 0) ? 4 : (RECW % 2 == 0) ? 2 : 1;
+    for (int i = lane * G; i < words; i += 32 * G) cp_async<4 * G>(dst + i, src + i);
+}
+
 struct MmaSmem {
-    uint32_t klut, klut_lo, slut, vlut, rowsc, stage, ptile, total;
-    uint32_t stage_bytes, kc, ks, vc, kn, kr, vn;
+    uint32_t klut, slut, vlut, rowsc, ptile, stage, total;
+    uint32_t stage_bytes, kc, ks, vc;
 };
 
 __host__ __device__ inline MmaSmem mma_smem_layout(int D, int KB, int VB, int m) {
     MmaSmem L;
     uint32_t o = 0;
     L.klut = o;
-    o += 64 * 4;
-    L.klut_lo = o;
-    o += 64 * 4;
+    o += 64 * 8;
     L.slut = o;
     o += 16 * 4;
     L.vlut = o;
     o += 64 * 4;
     L.rowsc = o;
-    o += 4 * kRowsPerCta * 4;
+    o += 2 * kRowsPerCta * 4;
     L.ptile = o;
     o += 4 * kRowsPerCta * 16 * 2;
     o = (o + 15) & ~15u;
     const uint32_t g32 = D / 32;
     L.kc = 0;
-    L.ks = L.kc + kStageTok * KB * g32 * 4;
-    L.vc = L.ks + kStageTok * (m / 32) * 4;
-    L.kn = L.vc + kStageTok * VB * g32 * 4;
-    L.kr = L.kn + kStageTok * 2;
-    L.vn = L.kr + kStageTok * 2;
-    L.stage_bytes = (L.vn + kStageTok * 2 + 15) & ~15u;
+    L.ks = L.kc + kWarpStage * KB * g32 * 4;
+    L.vc = L.ks + kWarpStage * (m / 32) * 4;
+    L.stage_bytes = (L.vc + kWarpStage * VB * g32 * 4 + 15) & ~15u;
     L.stage = o;
-    o += 2 * L.stage_bytes;
-    // the cross-warp combine reuses the stage buffers: 4 warps x 8 rows x (D + 2) floats
+    o += 4 * 2 * L.stage_bytes;  // 4 warps x 2 stages
     const uint32_t comb = 4u * kRowsPerCta * (D + 2) * 4;
     if (o < L.stage + comb) o = L.stage + comb;
     L.total = o;
     return L;
 }
 
-template <int D, int KB, int VB, bool ATTEND>
+template <int D, int KB, int VB, bool ATTEND, bool PACK4>
 __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, ScoreProblem sp,
                                                                  const float *__restrict__ qprep, float scale,
                                                                  float *__restrict__ out, int splits,
                                                                  int row_groups) {
     constexpr int G32 = D / 32;
     constexpr int KSTEP = D / 16;
+    constexpr int MSTEP = KSTEP / 2;  // proj_dim = head_dim / 2
+    constexpr int SW = MSTEP / 2;     // sign words per key
     constexpr int KWPT = KB * G32;
     constexpr int VWPT = VB * G32;
-    // Scores are always carried at split precision: with large key norms (outlier channels) a
-    // single fp16 product moves the softmax logits by more than the output tolerance allows.
-    constexpr bool SPLIT = true;
-    constexpr int MSTEP = KSTEP / 2;  // proj_dim = head_dim / 2
+    constexpr int KSH = (KB <= 2) ? 3 : 2;  // key pair index scaled by 8 (or 4, then doubled)
     const int m = P.m;
-    constexpr int SW = MSTEP / 2;
     const MmaSmem L = mma_smem_layout(D, KB, ATTEND ? VB : 0, m);
 
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *klut = (uint32_t *)(smem + L.klut);
-    uint32_t *klut_lo = (uint32_t *)(smem + L.klut_lo);
+    uint2 *klut = (uint2 *)(smem + L.klut);
     uint32_t *slut = (uint32_t *)(smem + L.slut);
     uint32_t *vlut = (uint32_t *)(smem + L.vlut);
-    float *rowsc = (float *)(smem + L.rowsc);  // [4][8]: q scale, sq scale, real row flag, spare
+    float *rowsc = (float *)(smem + L.rowsc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, t4 = lane & 3;
@@ -135,12 +170,17 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     const int r0 = rg * kRowsPerCta;
     const int nrows = min(kRowsPerCta, rows - r0);
     const int64_t chunk = (sp.T + splits - 1) / splits;
-    const int64_t t0 = (int64_t)split * chunk;
+    const int64_t t0 = min(sp.T, (int64_t)split * chunk);
     const int64_t t1 = min(sp.T, t0 + chunk);
     const int stride = P.d + m;
     const float gamma = sqrtf(1.5707963267948966f) / (float)m;
+    auto qrow_of = [&](int rr) {
+        const int row = r0 + rr;
+        const int g = row / sp.Nq, i = row % sp.Nq;
+        return ((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i;
+    };
 
-    // ---- codebook scales and pair look-up tables
+    // ---- pair look-up tables and per-row query scales
     float kmax = 0.f, vmax = 0.f;
     for (int k = 0; k < (1 << KB); ++k) kmax = fmaxf(kmax, fabsf(P.cb->kc[k]));
     if (ATTEND)
@@ -148,106 +188,101 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     const int ek = scale_exp(kmax), ev = scale_exp(vmax);
     const float ksc = ldexpf(1.f, ek), vsc = ldexpf(1.f, ev);
     for (int e = tid; e < (1 << (2 * KB)); e += kThreadsMma) {
-        // index bits: plane p of (coord j, coord j+1) at bits (2p, 2p+1)
+        // index bits: plane p of (coordinate j, coordinate j+1) at bits (2p, 2p+1)
         int i0 = 0, i1 = 0;
         for (int p = 0; p < KB; ++p) {
             i0 |= ((e >> (2 * p)) & 1) << p;
             i1 |= ((e >> (2 * p + 1)) & 1) << p;
         }
         const float a0 = P.cb->kc[i0] * ksc, a1 = P.cb->kc[i1] * ksc;
-        klut[e] = pack_h2(a0, a1);
-        const float h0 = __half2float(__float2half_rn(a0)), h1 = __half2float(__float2half_rn(a1));
-        klut_lo[e] = pack_h2(a0 - h0, a1 - h1);
+        klut[e] = make_uint2(pack_h2(a0, a1), pack_h2(a0 - hi_part(a0), a1 - hi_part(a1)));
     }
-    if (tid < 4) {
-        // sign pair: bit0 -> projection j, bit1 -> projection j+1; 1 -> +1, 0 -> -1
-        slut[tid] = pack_h2((tid & 1) ? 1.f : -1.f, (tid & 2) ? 1.f : -1.f);
-    }
+    if (tid < 4) slut[tid] = pack_h2((tid & 1) ? 1.f : -1.f, (tid & 2) ? 1.f : -1.f);
     if (ATTEND) {
         for (int e = tid; e < (1 << (2 * VB)); e += kThreadsMma) {
             // low VB bits: token 2i, next VB bits: token 2i+1 (same coordinate)
-            const float a0 = P.cb->vc[e & ((1 << VB) - 1)] * vsc, a1 = P.cb->vc[e >> VB] * vsc;
-            vlut[e] = pack_h2(a0, a1);
+            vlut[e] = pack_h2(P.cb->vc[e & ((1 << VB) - 1)] * vsc, P.cb->vc[e >> VB] * vsc);
         }
     }
-    // ---- per-row query scales and B fragments (row gid of this CTA's group)
     if (tid < kRowsPerCta) {
-        float qm = 0.f, sm_ = 0.f;
+        float qm = 0.f, smx = 0.f;
         if (tid < nrows) {
-            const int rr = r0 + tid;
-            const int g = rr / sp.Nq, i = rr % sp.Nq;
-            const int64_t qrow = ((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i;
-            const float *qp = qprep + qrow * stride;
+            const float *qp = qprep + qrow_of(tid) * stride;
             for (int j = 0; j < D; ++j) qm = fmaxf(qm, fabsf(qp[j]));
-            for (int a = 0; a < m; ++a) sm_ = fmaxf(sm_, fabsf(qp[D + a]));
+            for (int a = 0; a < m; ++a) smx = fmaxf(smx, fabsf(qp[D + a]));
         }
         rowsc[tid] = (float)scale_exp(qm);
-        rowsc[kRowsPerCta + tid] = (float)scale_exp(sm_);
+        rowsc[kRowsPerCta + tid] = (float)scale_exp(smx);
     }
+    uint16_t *ptile = (uint16_t *)(smem + L.ptile) + warp * (kRowsPerCta * 16);
+    for (int e = lane; e < kRowsPerCta * 16; e += 32) ptile[e] = 0;
     __syncthreads();
-    uint32_t bq[KSTEP][2], bql[KSTEP][2], bs[MSTEP][2], bsl[MSTEP][2];
+
+    // ---- B fragments (queries) in registers
+    // PACK4: column n = gid holds row (gid & 3), hi part for gid < 4 and lo part for gid >= 4.
+    uint32_t bq[KSTEP][2], bql[PACK4 ? 1 : KSTEP][2], bs[MSTEP][2], bsl[PACK4 ? 1 : MSTEP][2];
     {
-        const bool real = gid < nrows;
-        const float *qp = nullptr;
-        if (real) {
-            const int rr = r0 + gid;
-            const int g = rr / sp.Nq, i = rr % sp.Nq;
-            const int64_t qrow = ((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i;
-            qp = qprep + qrow * stride;
-        }
-        const float qs = ldexpf(1.f, (int)rowsc[gid]), ss = ldexpf(1.f, (int)rowsc[kRowsPerCta + gid]);
+        const int brow = PACK4 ? (gid & 3) : gid;
+        const bool lo_col = PACK4 && gid >= 4;
+        const bool real = brow < nrows;
+        const float *qp = real ? qprep + qrow_of(brow) * stride : nullptr;
+        const float qs = ldexpf(1.f, (int)rowsc[brow]), ss = ldexpf(1.f, (int)rowsc[kRowsPerCta + brow]);
 #pragma unroll
         for (int s = 0; s < KSTEP; ++s) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int j = 16 * s + 8 * h + 2 * t4;
-                float x0 = real ? qp[j] * qs : 0.f, x1 = real ? qp[j + 1] * qs : 0.f;
-                bq[s][h] = pack_h2(x0, x1);
-                bql[s][h] = pack_h2(x0 - __half2float(__float2half_rn(x0)), x1 - __half2float(__float2half_rn(x1)));
+                const float x0 = real ? qp[j] * qs : 0.f, x1 = real ? qp[j + 1] * qs : 0.f;
+                const float l0 = x0 - hi_part(x0), l1 = x1 - hi_part(x1);
+                bq[s][h] = lo_col ? pack_h2(l0, l1) : pack_h2(x0, x1);
+                if constexpr (!PACK4) bql[s][h] = pack_h2(l0, l1);
                 if (s < MSTEP) {
                     const float y0 = real ? qp[D + j] * ss : 0.f, y1 = real ? qp[D + j + 1] * ss : 0.f;
-                    bs[s < MSTEP ? s : 0][h] = pack_h2(y0, y1);
-                    bsl[s < MSTEP ? s : 0][h] =
-                        pack_h2(y0 - __half2float(__float2half_rn(y0)), y1 - __half2float(__float2half_rn(y1)));
+                    const float m0 = y0 - hi_part(y0), m1 = y1 - hi_part(y1);
+                    bs[s < MSTEP ? s : 0][h] = lo_col ? pack_h2(m0, m1) : pack_h2(y0, y1);
+                    if constexpr (!PACK4) bsl[s < MSTEP ? s : 0][h] = pack_h2(m0, m1);
                 }
             }
         }
     }
-    // unscale factors of the thread's two accumulator rows (2*t4, 2*t4+1)
-    const float qun0 = ldexpf(1.f, -(int)rowsc[2 * t4] - ek), qun1 = ldexpf(1.f, -(int)rowsc[2 * t4 + 1] - ek);
-    const float sun0 = ldexpf(1.f, -(int)rowsc[kRowsPerCta + 2 * t4]);
-    const float sun1 = ldexpf(1.f, -(int)rowsc[kRowsPerCta + 2 * t4 + 1]);
+    // accumulator rows of this thread: (2*t4, 2*t4+1), or (2*(t4&1), +1) once PACK4 halves are summed
+    const int ra = PACK4 ? 2 * (t4 & 1) : 2 * t4;
+    const float qun0 = ldexpf(1.f, -(int)rowsc[ra] - ek), qun1 = ldexpf(1.f, -(int)rowsc[ra + 1] - ek);
+    const float sun0 = ldexpf(1.f, -(int)rowsc[kRowsPerCta + ra]);
+    const float sun1 = ldexpf(1.f, -(int)rowsc[kRowsPerCta + ra + 1]);
+    const bool writes_p = !PACK4 || t4 < 2;
 
-    // ---- token stages
-    uint8_t *stage0 = smem + L.stage;
-    auto stage_ptr = [&](int s) { return stage0 + (s & 1) * L.stage_bytes; };
+    // ---- this warp's token range and stage ring
+    const int64_t wlen = (((t1 - t0) + 4 * 16 - 1) / (4 * 16)) * 16;
+    const int64_t wt0 = min(t1, t0 + warp * wlen);
+    const int64_t wt1 = min(t1, wt0 + wlen);
+    uint8_t *wstage = smem + L.stage + (size_t)warp * 2 * L.stage_bytes;
     const int64_t rec_base = sl * sp.T;
-    uint16_t nk_reg = 0, nr_reg = 0, nv_reg = 0;
-    auto issue = [&](int s, int64_t tb) {
-        if (tb < t1) {
-            const int ntok = (int)min((int64_t)kStageTok, t1 - tb);
-            uint8_t *st = stage_ptr(s);
+    auto issue = [&](int s) {
+        const int64_t tb = wt0 + (int64_t)s * kWarpStage;
+        if (tb < wt1) {
+            const int ntok = (int)min((int64_t)kWarpStage, wt1 - tb);
+            uint8_t *st = wstage + (s & 1) * L.stage_bytes;
             const int64_t rec0 = rec_base + tb;
-            uint32_t *dkc = (uint32_t *)(st + L.kc);
-            const uint32_t *gkc = sp.kcodes + rec0 * KWPT;
-            for (int i = tid; i < ntok * KWPT; i += kThreadsMma) cp_async4(dkc + i, gkc + i);
-            uint32_t *dks = (uint32_t *)(st + L.ks);
-            const uint32_t *gks = sp.ksigns + rec0 * SW;
-            for (int i = tid; i < ntok * SW; i += kThreadsMma) cp_async4(dks + i, gks + i);
-            if (ATTEND) {
-                uint32_t *dvc = (uint32_t *)(st + L.vc);
-                const uint32_t *gvc = sp.vcodes + rec0 * VWPT;
-                for (int i = tid; i < ntok * VWPT; i += kThreadsMma) cp_async4(dvc + i, gvc + i);
-            }
+            stage_copy<KWPT>((uint32_t *)(st + L.kc), sp.kcodes + rec0 * KWPT, ntok * KWPT, lane);
+            stage_copy<SW>((uint32_t *)(st + L.ks), sp.ksigns + rec0 * SW, ntok * SW, lane);
+            if (ATTEND) stage_copy<VWPT>((uint32_t *)(st + L.vc), sp.vcodes + rec0 * VWPT, ntok * VWPT, lane);
         }
         cp_async_commit();
     };
-    auto load_norms = [&](int64_t tb) {
-        if (tb < t1 && tid < min((int64_t)kStageTok, t1 - tb)) {
-            const int64_t rec = rec_base + tb + tid;
-            nk_reg = sp.knorm[rec];
-            nr_reg = sp.krnorm[rec];
-            if (ATTEND) nv_reg = sp.vnorm[rec];
+    // norms of the thread's two tokens (gid, gid+8) of a 16-token block
+    float nka = 0.f, nkb = 0.f, nra = 0.f, nrb = 0.f, nva = 0.f, nvb = 0.f;
+    auto load_norms = [&](int64_t gtb) {
+        const int64_t ta = gtb + gid, tb = gtb + gid + 8;
+        if (ta < wt1) {
+            nka = f16_bits_to_f32(sp.knorm[rec_base + ta]);
+            nra = f16_bits_to_f32(sp.krnorm[rec_base + ta]);
+            if (ATTEND) nva = f16_bits_to_f32(sp.vnorm[rec_base + ta]);
+        }
+        if (tb < wt1) {
+            nkb = f16_bits_to_f32(sp.knorm[rec_base + tb]);
+            nrb = f16_bits_to_f32(sp.krnorm[rec_base + tb]);
+            if (ATTEND) nvb = f16_bits_to_f32(sp.vnorm[rec_base + tb]);
         }
     };
 
@@ -255,105 +290,106 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
 #pragma unroll
     for (int c = 0; c < (ATTEND ? KSTEP : 1); ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
     float M0 = -INFINITY, M1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    uint16_t *ptile = (uint16_t *)(smem + L.ptile) + warp * (kRowsPerCta * 16);
 
-    issue(0, t0);
-    issue(1, t0 + kStageTok);
-    load_norms(t0);
-    int s = 0;
-    for (int64_t tb = t0; tb < t1; tb += kStageTok, ++s) {
-        uint8_t *st = stage_ptr(s);
+    const int nstages = (int)((wt1 - wt0 + kWarpStage - 1) / kWarpStage);
+    issue(0);
+    issue(1);
+    load_norms(wt0);
+    for (int s = 0; s < nstages; ++s) {
         cp_async_wait<1>();
-        {
-            uint16_t *kn_s = (uint16_t *)(st + L.kn), *kr_s = (uint16_t *)(st + L.kr), *vn_s = (uint16_t *)(st + L.vn);
-            kn_s[tid] = nk_reg;
-            kr_s[tid] = nr_reg;
-            if (ATTEND) vn_s[tid] = nv_reg;
-        }
-        __syncthreads();
-        load_norms(tb + kStageTok);
-        const int ntok = (int)min((int64_t)kStageTok, t1 - tb);
+        __syncwarp();
+        const uint8_t *st = wstage + (s & 1) * L.stage_bytes;
         const uint32_t *skc = (const uint32_t *)(st + L.kc);
         const uint32_t *sks = (const uint32_t *)(st + L.ks);
         const uint32_t *svc = (const uint32_t *)(st + L.vc);
-        const uint16_t *skn = (const uint16_t *)(st + L.kn);
-        const uint16_t *skr = (const uint16_t *)(st + L.kr);
-        const uint16_t *svn = (const uint16_t *)(st + L.vn);
-        for (int blk = warp; blk * 16 < ntok; blk += 4) {
-            const int ob = blk * 16;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            const int ob = 16 * half;
+            const int64_t gtb = wt0 + (int64_t)s * kWarpStage + ob;
+            if (gtb >= wt1) break;
             const int ta = ob + gid, tb8 = ob + gid + 8;
-            const bool va = ta < ntok, vb = tb8 < ntok;
+            const bool va = gtb + gid < wt1, vb = gtb + gid + 8 < wt1;
+            const float kna = nka, knb = nkb, rna = nra * gamma, rnb = nrb * gamma, vna = nva, vnb = nvb;
+            load_norms(gtb + 16);  // next block's norms, in flight during this block
             // ---------------- scores
             float cs[4] = {0.f, 0.f, 0.f, 0.f}, cd[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                uint32_t wa[KWPT], wb[KWPT];
+                load_words<KWPT>(skc + ta * KWPT, wa);
+                load_words<KWPT>(skc + tb8 * KWPT, wb);
 #pragma unroll
-            for (int g = 0; g < G32; ++g) {
-                uint32_t ya = 0, yb = 0;
+                for (int g = 0; g < G32; ++g) {
+                    uint32_t ya = 0, yb = 0;
 #pragma unroll
-                for (int p = 0; p < KB; ++p) {
-                    ya |= ((skc[ta * KWPT + g * KB + p] >> (2 * t4)) & 0x03030303u) << (2 * p + 2);
-                    yb |= ((skc[tb8 * KWPT + g * KB + p] >> (2 * t4)) & 0x03030303u) << (2 * p + 2);
-                }
+                    for (int p = 0; p < KB; ++p) {
+                        ya |= ((wa[g * KB + p] >> (2 * t4)) & 0x03030303u) << (2 * p + KSH);
+                        yb |= ((wb[g * KB + p] >> (2 * t4)) & 0x03030303u) << (2 * p + KSH);
+                    }
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int sh0 = 16 * h, sh1 = 16 * h + 8;
-                    uint32_t a[4];
-                    a[0] = lut_at(klut, (ya >> sh0) & 0xFFu);
-                    a[1] = lut_at(klut, (yb >> sh0) & 0xFFu);
-                    a[2] = lut_at(klut, (ya >> sh1) & 0xFFu);
-                    a[3] = lut_at(klut, (yb >> sh1) & 0xFFu);
-                    mma16816(cs, a, bq[2 * g + h][0], bq[2 * g + h][1]);
-                    if (SPLIT) {
-                        uint32_t al[4];
-                        al[0] = lut_at(klut_lo, (ya >> sh0) & 0xFFu);
-                        al[1] = lut_at(klut_lo, (yb >> sh0) & 0xFFu);
-                        al[2] = lut_at(klut_lo, (ya >> sh1) & 0xFFu);
-                        al[3] = lut_at(klut_lo, (yb >> sh1) & 0xFFu);
-                        mma16816(cs, a, bql[2 * g + h][0], bql[2 * g + h][1]);
-                        mma16816(cs, al, bq[2 * g + h][0], bq[2 * g + h][1]);
+                    for (int h = 0; h < 2; ++h) {
+                        const int sh0 = 16 * h, sh1 = 16 * h + 8;
+                        uint32_t o[4] = {(ya >> sh0) & 0xFFu, (yb >> sh0) & 0xFFu, (ya >> sh1) & 0xFFu,
+                                         (yb >> sh1) & 0xFFu};
+                        uint32_t ah[4], al[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint2 e = lut64(klut, KSH == 3 ? o[u] : (o[u] << 1));
+                            ah[u] = e.x;
+                            al[u] = e.y;
+                        }
+                        mma16816(cs, ah, bq[2 * g + h][0], bq[2 * g + h][1]);
+                        if constexpr (PACK4) {
+                            mma16816(cs, al, bq[2 * g + h][0], bq[2 * g + h][1]);
+                        } else {
+                            mma16816(cs, ah, bql[2 * g + h][0], bql[2 * g + h][1]);
+                            mma16816(cs, al, bq[2 * g + h][0], bq[2 * g + h][1]);
+                        }
                     }
                 }
-            }
+                uint32_t sa[SW], sb[SW];
+                load_words<SW>(sks + ta * SW, sa);
+                load_words<SW>(sks + tb8 * SW, sb);
 #pragma unroll
-            for (int g = 0; g < SW; ++g) {
-                {
-                    const uint32_t ya = ((sks[ta * SW + g] >> (2 * t4)) & 0x03030303u) << 2;
-                    const uint32_t yb = ((sks[tb8 * SW + g] >> (2 * t4)) & 0x03030303u) << 2;
+                for (int g = 0; g < SW; ++g) {
+                    const uint32_t ya = ((sa[g] >> (2 * t4)) & 0x03030303u) << 2;
+                    const uint32_t yb = ((sb[g] >> (2 * t4)) & 0x03030303u) << 2;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int sh0 = 16 * h, sh1 = 16 * h + 8;
                         uint32_t a[4];
-                        a[0] = lut_at(slut, (ya >> sh0) & 0xFFu);
-                        a[1] = lut_at(slut, (yb >> sh0) & 0xFFu);
-                        a[2] = lut_at(slut, (ya >> sh1) & 0xFFu);
-                        a[3] = lut_at(slut, (yb >> sh1) & 0xFFu);
+                        a[0] = lut32(slut, (ya >> sh0) & 0xFFu);
+                        a[1] = lut32(slut, (yb >> sh0) & 0xFFu);
+                        a[2] = lut32(slut, (ya >> sh1) & 0xFFu);
+                        a[3] = lut32(slut, (yb >> sh1) & 0xFFu);
                         mma16816(cd, a, bs[2 * g + h][0], bs[2 * g + h][1]);
-                        if (SPLIT) mma16816(cd, a, bsl[2 * g + h][0], bsl[2 * g + h][1]);
+                        if constexpr (!PACK4) mma16816(cd, a, bsl[2 * g + h][0], bsl[2 * g + h][1]);
                     }
                 }
             }
-            const float kna = f16_bits_to_f32(skn[ta]), knb = f16_bits_to_f32(skn[tb8]);
-            const float rna = f16_bits_to_f32(skr[ta]) * gamma, rnb = f16_bits_to_f32(skr[tb8]) * gamma;
+            if constexpr (PACK4) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    cs[e] += __shfl_xor_sync(kFull, cs[e], 2);
+                    cd[e] += __shfl_xor_sync(kFull, cd[e], 2);
+                }
+            }
             float sc[4];
             sc[0] = kna * fmaf(rna, cd[0] * sun0, cs[0] * qun0);
             sc[1] = kna * fmaf(rna, cd[1] * sun1, cs[1] * qun1);
             sc[2] = knb * fmaf(rnb, cd[2] * sun0, cs[2] * qun0);
             sc[3] = knb * fmaf(rnb, cd[3] * sun1, cs[3] * qun1);
-            if (!ATTEND) {
-                // raw scores out: rows 2*t4, 2*t4+1 of this group, tokens ta, tb8
+            if constexpr (!ATTEND) {
+                if (writes_p) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int rr = 2 * t4 + (e & 1);
-                    const bool v = (e < 2) ? va : vb;
-                    if (v && rr < nrows) {
-                        const int row = r0 + rr;
-                        const int g = row / sp.Nq, i = row % sp.Nq;
-                        const int64_t qrow = ((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i;
-                        out[qrow * sp.T + tb + ((e < 2) ? ta : tb8)] = sc[e];
+                    for (int e = 0; e < 4; ++e) {
+                        const int rr = ra + (e & 1);
+                        const bool v = (e < 2) ? va : vb;
+                        if (v && rr < nrows) out[qrow_of(rr) * sp.T + gtb + ((e < 2) ? gid : gid + 8)] = sc[e];
                     }
                 }
                 continue;
             }
-            // ---------------- online softmax (rows 2*t4, 2*t4+1)
+            // ---------------- online softmax (rows ra, ra+1)
             const float z0 = va ? scale * sc[0] : -INFINITY, z1 = va ? scale * sc[1] : -INFINITY;
             const float z2 = vb ? scale * sc[2] : -INFINITY, z3 = vb ? scale * sc[3] : -INFINITY;
             float bm0 = fmaxf(z0, z2), bm1 = fmaxf(z1, z3);
@@ -380,49 +416,58 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
                     oacc[c][3] *= al1;
                 }
             }
-            // probabilities times value norms, transposed through shared memory
-            const float vna = va ? f16_bits_to_f32(svn[ta]) : 0.f, vnb = vb ? f16_bits_to_f32(svn[tb8]) : 0.f;
-            ptile[(2 * t4) * 16 + gid] = __half_as_ushort(__float2half_rn(p0 * vna));
-            ptile[(2 * t4 + 1) * 16 + gid] = __half_as_ushort(__float2half_rn(p1 * vna));
-            ptile[(2 * t4) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(p2 * vnb));
-            ptile[(2 * t4 + 1) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(p3 * vnb));
+            // probabilities times value norms, transposed through shared memory (rows >= 4 of
+            // the tile stay zero in PACK4 mode)
+            if (writes_p) {
+                const float pa = va ? vna : 0.f, pb = vb ? vnb : 0.f;
+                ptile[ra * 16 + gid] = __half_as_ushort(__float2half_rn(p0 * pa));
+                ptile[(ra + 1) * 16 + gid] = __half_as_ushort(__float2half_rn(p1 * pa));
+                ptile[ra * 16 + gid + 8] = __half_as_ushort(__float2half_rn(p2 * pb));
+                ptile[(ra + 1) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(p3 * pb));
+            }
             __syncwarp();
             const uint32_t bp0 = *(const uint32_t *)(ptile + gid * 16 + 2 * t4);
             const uint32_t bp1 = *(const uint32_t *)(ptile + gid * 16 + 2 * t4 + 8);
             __syncwarp();
-            // ---------------- values: A = Vhat^T (coords x tokens), pairs along tokens
-            const int tk0 = ob + 2 * t4, tk8 = ob + 2 * t4 + 8;
+            // ---------------- values: A = Vhat^T (coordinates x tokens), pairs along tokens
+            {
+                uint32_t v0[VWPT], v1[VWPT], v8[VWPT], v9[VWPT];
+                const int tk = ob + 2 * t4;
+                load_words<VWPT>(svc + tk * VWPT, v0);
+                load_words<VWPT>(svc + (tk + 1) * VWPT, v1);
+                load_words<VWPT>(svc + (tk + 8) * VWPT, v8);
+                load_words<VWPT>(svc + (tk + 9) * VWPT, v9);
 #pragma unroll
-            for (int g = 0; g < G32; ++g) {
-                uint32_t z[4];
+                for (int g = 0; g < G32; ++g) {
+                    uint32_t z0w = 0, z1w = 0, z8w = 0, z9w = 0;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int tt = ((u & 2) ? tk8 : tk0) + (u & 1);
-                    uint32_t acc = 0;
+                    for (int p = 0; p < VB; ++p) {
+                        z0w |= ((v0[g * VB + p] >> gid) & 0x01010101u) << p;
+                        z1w |= ((v1[g * VB + p] >> gid) & 0x01010101u) << p;
+                        z8w |= ((v8[g * VB + p] >> gid) & 0x01010101u) << p;
+                        z9w |= ((v9[g * VB + p] >> gid) & 0x01010101u) << p;
+                    }
+                    const uint32_t zz01 = (z0w << 2) | (z1w << (VB + 2));
+                    const uint32_t zz89 = (z8w << 2) | (z9w << (VB + 2));
 #pragma unroll
-                    for (int p = 0; p < VB; ++p) acc |= ((svc[tt * VWPT + g * VB + p] >> gid) & 0x01010101u) << p;
-                    z[u] = acc;
-                }
-                const uint32_t zz01 = (z[0] << 2) | (z[1] << (VB + 2));
-                const uint32_t zz89 = (z[2] << 2) | (z[3] << (VB + 2));
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t a[4];
-                    a[0] = lut_at(vlut, (zz01 >> (16 * h)) & 0xFFu);
-                    a[1] = lut_at(vlut, (zz01 >> (16 * h + 8)) & 0xFFu);
-                    a[2] = lut_at(vlut, (zz89 >> (16 * h)) & 0xFFu);
-                    a[3] = lut_at(vlut, (zz89 >> (16 * h + 8)) & 0xFFu);
-                    mma16816(oacc[2 * g + h], a, bp0, bp1);
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t a[4];
+                        a[0] = lut32(vlut, (zz01 >> (16 * h)) & 0xFFu);
+                        a[1] = lut32(vlut, (zz01 >> (16 * h + 8)) & 0xFFu);
+                        a[2] = lut32(vlut, (zz89 >> (16 * h)) & 0xFFu);
+                        a[3] = lut32(vlut, (zz89 >> (16 * h + 8)) & 0xFFu);
+                        mma16816(oacc[2 * g + h], a, bp0, bp1);
+                    }
                 }
             }
         }
-        __syncthreads();
-        issue(s + 2, tb + 2 * kStageTok);
+        __syncwarp();
+        issue(s + 2);
     }
     cp_async_wait<0>();
-    if (!ATTEND) return;
+    if constexpr (!ATTEND) return;
 
-    // ---- combine the four warps' partial softmax states, write (M, L, o_rot) per row
+    // ---- merge the four warps' softmax states, write (M, L, o_rot) per row
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
         l0 += __shfl_xor_sync(kFull, l0, o);
@@ -433,19 +478,21 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     const float ounsc = ldexpf(1.f, -ev);
     {
         float *cw = comb + (size_t)warp * kRowsPerCta * (D + 2);
-        if (gid == 0) {
-            cw[(2 * t4) * (D + 2)] = M0;
-            cw[(2 * t4) * (D + 2) + 1] = l0;
-            cw[(2 * t4 + 1) * (D + 2)] = M1;
-            cw[(2 * t4 + 1) * (D + 2) + 1] = l1;
+        if (gid == 0 && writes_p) {
+            cw[ra * (D + 2)] = M0;
+            cw[ra * (D + 2) + 1] = l0;
+            cw[(ra + 1) * (D + 2)] = M1;
+            cw[(ra + 1) * (D + 2) + 1] = l1;
         }
+        if (writes_p) {
 #pragma unroll
-        for (int c = 0; c < KSTEP; ++c) {
-            const int j0 = 16 * c + gid, j1 = j0 + 8;
-            cw[(2 * t4) * (D + 2) + 2 + j0] = oacc[c][0] * ounsc;
-            cw[(2 * t4 + 1) * (D + 2) + 2 + j0] = oacc[c][1] * ounsc;
-            cw[(2 * t4) * (D + 2) + 2 + j1] = oacc[c][2] * ounsc;
-            cw[(2 * t4 + 1) * (D + 2) + 2 + j1] = oacc[c][3] * ounsc;
+            for (int c = 0; c < KSTEP; ++c) {
+                const int j0 = 16 * c + gid, j1 = j0 + 8;
+                cw[(2 * t4) * (D + 2) + 2 + j0] = oacc[c][0] * ounsc;
+                cw[(2 * t4 + 1) * (D + 2) + 2 + j0] = oacc[c][1] * ounsc;
+                cw[(2 * t4) * (D + 2) + 2 + j1] = oacc[c][2] * ounsc;
+                cw[(2 * t4 + 1) * (D + 2) + 2 + j1] = oacc[c][3] * ounsc;
+            }
         }
     }
     __syncthreads();
@@ -466,20 +513,17 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
                 v = fmaf(f, comb[(w * kRowsPerCta + rr) * (D + 2) + col], v);
             }
         }
-        const int row = r0 + rr;
-        const int g = row / sp.Nq, i = row % sp.Nq;
-        const int64_t qrow = ((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i;
-        out[(qrow * splits + split) * (int64_t)(D + 2) + col] = v;
+        out[(qrow_of(rr) * splits + split) * (int64_t)(D + 2) + col] = v;
     }
 }
 
-template <int D, int KB, int VB, bool ATTEND>
+template <int D, int KB, int VB, bool ATTEND, bool PACK4>
 cudaError_t launch_dm(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale, float *out,
                       int splits, cudaStream_t s) {
     const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
     const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
     const MmaSmem L = mma_smem_layout(D, KB, ATTEND ? VB : 0, P.m);
-    auto kern = decode_mma_kernel<D, KB, VB, ATTEND>;
+    auto kern = decode_mma_kernel<D, KB, VB, ATTEND, PACK4>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)splits, (unsigned)((int64_t)sp.B * sp.Hkv * row_groups));
@@ -487,18 +531,26 @@ cudaError_t launch_dm(const Prepared &P, const ScoreProblem &sp, const float *qp
     return cudaGetLastError();
 }
 
+template <int D, int KB, int VB, bool ATTEND>
+cudaError_t launch_dm_pack(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale, float *out,
+                           int splits, cudaStream_t s) {
+    const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
+    if (rows <= 4) return launch_dm<D, KB, VB, ATTEND, true>(P, sp, qprep, scale, out, splits, s);
+    return launch_dm<D, KB, VB, ATTEND, false>(P, sp, qprep, scale, out, splits, s);
+}
+
 template <int D, bool ATTEND>
 cudaError_t launch_dm_bits(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale, float *out,
                            int splits, cudaStream_t s) {
     const int kb = P.kbeta, vb = P.vbeta;
     if constexpr (ATTEND) {
-        if (kb == 1 && vb == 2) return launch_dm<D, 1, 2, true>(P, sp, qprep, scale, out, splits, s);
-        if (kb == 2 && vb == 3) return launch_dm<D, 2, 3, true>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 1 && vb == 2) return launch_dm_pack<D, 1, 2, true>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 2 && vb == 3) return launch_dm_pack<D, 2, 3, true>(P, sp, qprep, scale, out, splits, s);
     } else {
         // scores only: the value bit width is irrelevant
-        if (kb == 1) return launch_dm<D, 1, 1, false>(P, sp, qprep, scale, out, splits, s);
-        if (kb == 2) return launch_dm<D, 2, 1, false>(P, sp, qprep, scale, out, splits, s);
-        if (kb == 3) return launch_dm<D, 3, 1, false>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 1) return launch_dm_pack<D, 1, 1, false>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 2) return launch_dm_pack<D, 2, 1, false>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 3) return launch_dm_pack<D, 3, 1, false>(P, sp, qprep, scale, out, splits, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -511,20 +563,15 @@ bool decode_mma_supported(const Prepared &P, const ScoreProblem &sp, bool attend
     const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
     if (!attend && rows > 64) return false;
     const int kb = P.kbeta, vb = P.vbeta;
-    if (attend) {
-        const bool ok = (kb == 1 && vb == 2) || (kb == 2 && vb == 3);
-        if (!ok) return false;
-    } else {
-        if (kb < 1 || kb > 3) return false;
-    }
-    return true;
+    if (attend) return (kb == 1 && vb == 2) || (kb == 2 && vb == 3);
+    return kb >= 1 && kb <= 3;
 }
 
 int decode_mma_splits(const ScoreProblem &sp) {
     const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
     const int64_t ctas = (int64_t)sp.B * sp.Hkv * ((rows + kRowsPerCta - 1) / kRowsPerCta);
     int64_t want = (148 * 8 + ctas - 1) / ctas;
-    int64_t cap = (sp.T + 2 * kStageTok - 1) / (2 * kStageTok);
+    int64_t cap = (sp.T + 4 * 2 * kWarpStage - 1) / (4 * 2 * kWarpStage);
     if (want > cap) want = cap;
     if (want < 1) want = 1;
     return (int)want;
