@@ -351,6 +351,126 @@ def run_tq(args):
     return 0
 
 
+def run_workload(args):
+    """Secondary measurements of the other workloads (one JSON line each, not the headline):
+    per-op device time with CUDA events after warm-up, rates, and HBM fractions."""
+    import numpy as np
+    import torch
+    from kv_cache_vector_compress_b200 import synth, tq
+    torch.cuda.set_device(0)
+    pk = peaks()
+    wl = args.workload
+    s = synth.seeds(wl)
+    st = torch.cuda.current_stream()
+
+    def timed(fn, steps=args.steps, warmup=args.warmup):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(steps):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    def rec(op, ms, units, unit, nbytes):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"op": op, "ms": ms, "units": units, f"{unit}_per_s": units / (ms * 1e-3), "GB/s": gbs,
+                "frac_hbm": gbs / pk["hbm_gbs"]}
+
+    out = []
+    if wl == 1:
+        w = synth.workload1()
+        d, m, bits, T = 128, 64, 3, 4096
+        p = tq.Params(d, bits, m, torch.from_numpy(w["R"]).cuda(), torch.from_numpy(w["S"]).cuda())
+        K, V, Q = (torch.from_numpy(w[k]).cuda() for k in ("K", "V", "Q"))
+        keys = tq.tq_compress_keys(p, K)
+        vals = tq.tq_compress_values(p, V)
+        ms = timed(lambda: tq.tq_compress_keys(p, K, *keys))
+        out.append(rec("compress_keys", ms, T, "vectors", T * (d * 4 + 44)))
+        ms = timed(lambda: tq.tq_compress_values(p, V, *vals))
+        out.append(rec("compress_values", ms, T, "vectors", T * (d * 4 + 50)))
+        sc = torch.empty((1, 1, 16, T), dtype=torch.float32, device="cuda")
+        ms = timed(lambda: tq.tq_scores(p, Q, keys, 1, T, scores=sc))
+        out.append(rec("scores", ms, T, "keys", T * 44 + 16 * T * 4))
+        o = torch.empty((1, 1, 16, d), dtype=torch.float32, device="cuda")
+        ms = timed(lambda: tq.tq_attend(p, Q, keys, vals, 1, T, out=o))
+        out.append(rec("attend", ms, T, "keys", T * 94))
+        name = "single head d128 3-bit: 4096 K + 4096 V fp32 unit vectors, 16 queries (latency)"
+    elif wl == 2:
+        d, m, L, H, T = 128, 64, 36, 2, 8192
+        n = L * H * T
+        R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
+        S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
+        sc = np.exp(np.random.Generator(np.random.PCG64(s["scales"])).standard_normal((L * H, d)))
+        K = (synth.torch_normal_f16((L * H, T, d), s["keys"]).float()
+             * torch.from_numpy(sc.astype(np.float32)).cuda()[:, None, :]).half().view(n, d)
+        V = synth.torch_normal_f16((n, d), s["values"])
+        for bits in (2, 3, 4):
+            p = tq.Params(d, bits, m, R, S)
+            keys = tq.tq_compress_keys(p, K)
+            vals = tq.tq_compress_values(p, V)
+            kb = (bits - 1) * d // 8 + m // 8 + 4
+            vb = bits * d // 8 + 2
+            ms = timed(lambda: tq.tq_compress_keys(p, K, *keys))
+            out.append(rec(f"compress_keys_b{bits}", ms, n, "vectors", n * (2 * d + kb)))
+            ms = timed(lambda: tq.tq_compress_values(p, V, *vals))
+            out.append(rec(f"compress_values_b{bits}", ms, n, "vectors", n * (2 * d + vb)))
+        name = "Qwen2.5-3B-shaped prefill compress: 36 layers x 2 KV heads x 8192 x 128 fp16, bits 2/3/4"
+    elif wl == 4:
+        d, m, B, Hq, Hkv, T = 256, 128, 8, 16, 4, 65536
+        n = B * Hkv * T
+        R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
+        S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
+        K = synth.torch_normal_f16((n, d), s["keys"])
+        K[:, torch.from_numpy(synth.outlier_channels(d, s["scales"])).cuda()] *= 20
+        V = synth.torch_normal_f16((n, d), s["values"])
+        Q = synth.torch_normal_f32((B, Hq, 1, d), s["queries"])
+        for bits in (2, 4):
+            p = tq.Params(d, bits, m, R, S)
+            keys = tq.tq_compress_keys(p, K)
+            vals = tq.tq_compress_values(p, V)
+            kb = (bits - 1) * d // 8 + m // 8 + 4
+            vb = bits * d // 8 + 2
+            ms = timed(lambda: tq.tq_compress_keys(p, K, *keys), steps=3)
+            out.append(rec(f"compress_keys_b{bits}", ms, n, "vectors", n * (2 * d + kb)))
+            ms = timed(lambda: tq.tq_compress_values(p, V, *vals), steps=3)
+            out.append(rec(f"compress_values_b{bits}", ms, n, "vectors", n * (2 * d + vb)))
+            o = torch.empty((B, Hq, 1, d), dtype=torch.float32, device="cuda")
+            scr = torch.empty(tq.tq_attend_scratch_bytes(p, B, Hq, Hkv, 1, T), dtype=torch.uint8, device="cuda")
+            ms = timed(lambda: tq.tq_attend(p, Q, keys, vals, Hkv, T, out=o, scratch=scr))
+            out.append(rec(f"attend_b{bits}", ms, n, "keys", n * (kb + vb)))
+        name = "wide-head decode: B8 Hq16/Hkv4 T65536 d256 m128, bits 2 and 4, 1% key channels x20"
+    elif wl == 5:
+        d, m, bits, N, Nq, k = 1024, 512, 4, 1_000_000, 1024, 10
+        R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
+        S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
+        p = tq.Params(d, bits, m, R, S)
+        X = synth.torch_normal_f32((N, d), s["keys"])
+        X /= X.norm(dim=1, keepdim=True)
+        Qv = synth.torch_normal_f32((1, 1, Nq, d), s["queries"])
+        Qv /= Qv.norm(dim=-1, keepdim=True)
+        keys = tq.tq_compress_keys(p, X)
+        kb = (bits - 1) * d // 8 + m // 8 + 4
+        ms = timed(lambda: tq.tq_compress_keys(p, X, *keys), steps=2, warmup=1)
+        out.append(rec("compress_db", ms, N, "vectors", N * (4 * d + kb)))
+        ti = torch.empty((1, 1, Nq, k), dtype=torch.int32, device="cuda")
+        tv = torch.empty((1, 1, Nq, k), dtype=torch.float32, device="cuda")
+        scr = torch.empty(tq.tq_scores_scratch_bytes(p, 1, 1, 1, Nq, N, k), dtype=torch.uint8, device="cuda")
+        ms = timed(lambda: tq.tq_scores(p, Qv, keys, 1, N, want_scores=False, topk=k, topk_idx=ti, topk_val=tv,
+                                        scratch=scr), steps=1, warmup=1)
+        r = rec("scores_top10", ms, N * Nq, "query_key_pairs", N * kb)
+        r["tflops_equiv"] = 2.0 * Nq * N * (d + m) / (ms * 1e-3) / 1e12
+        out.append(r)
+        name = "vector search: 1M x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
+    else:
+        raise SystemExit("unknown workload")
+    print(json.dumps({"workload": wl, "name": name, "ops": out, "peak_hbm_gbs": pk["hbm_gbs"]}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -359,9 +479,13 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's 32)")
+    ap.add_argument("--workload", type=int, default=3,
+                    help="3 (default) prints the headline line; 1, 2, 4, 5 print secondary per-op measurements")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != 3:
+        return run_workload(args)
     return run_tq(args)
 
 

@@ -119,11 +119,11 @@ __host__ __device__ inline MmaSmem mma_smem_layout(int D, int KB, int VB, int m)
     L.slut = o;
     o += 16 * 4;
     L.vlut = o;
-    o += 64 * 4;
+    o += 256 * 8;
     L.rowsc = o;
     o += 2 * kRowsPerCta * 4;
     L.ptile = o;
-    o += 4 * kRowsPerCta * 16 * 2;
+    o += 2 * 4 * kRowsPerCta * 16 * 2;  // per warp: P hi tile and P lo tile
     o = (o + 15) & ~15u;
     const uint32_t g32 = D / 32;
     L.kc = 0;
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     extern __shared__ __align__(16) uint8_t smem[];
     uint2 *klut = (uint2 *)(smem + L.klut);
     uint32_t *slut = (uint32_t *)(smem + L.slut);
-    uint32_t *vlut = (uint32_t *)(smem + L.vlut);
+    uint2 *vlut = (uint2 *)(smem + L.vlut);
     float *rowsc = (float *)(smem + L.rowsc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -200,8 +200,9 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     if (tid < 4) slut[tid] = pack_h2((tid & 1) ? 1.f : -1.f, (tid & 2) ? 1.f : -1.f);
     if (ATTEND) {
         for (int e = tid; e < (1 << (2 * VB)); e += kThreadsMma) {
-            // low VB bits: token 2i, next VB bits: token 2i+1 (same coordinate)
-            vlut[e] = pack_h2(P.cb->vc[e & ((1 << VB) - 1)] * vsc, P.cb->vc[e >> VB] * vsc);
+            // low VB bits: token 2i, next VB bits: token 2i+1 (same coordinate); hi and lo fp16 parts
+            const float a0 = P.cb->vc[e & ((1 << VB) - 1)] * vsc, a1 = P.cb->vc[e >> VB] * vsc;
+            vlut[e] = make_uint2(pack_h2(a0, a1), pack_h2(a0 - hi_part(a0), a1 - hi_part(a1)));
         }
     }
     if (tid < kRowsPerCta) {
@@ -214,8 +215,9 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
         rowsc[tid] = (float)scale_exp(qm);
         rowsc[kRowsPerCta + tid] = (float)scale_exp(smx);
     }
-    uint16_t *ptile = (uint16_t *)(smem + L.ptile) + warp * (kRowsPerCta * 16);
-    for (int e = lane; e < kRowsPerCta * 16; e += 32) ptile[e] = 0;
+    uint16_t *ptile = (uint16_t *)(smem + L.ptile) + warp * (2 * kRowsPerCta * 16);
+    uint16_t *ptile_lo = ptile + kRowsPerCta * 16;
+    for (int e = lane; e < 2 * kRowsPerCta * 16; e += 32) ptile[e] = 0;
     __syncthreads();
 
     // ---- B fragments (queries) in registers
@@ -416,47 +418,98 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
                     oacc[c][3] *= al1;
                 }
             }
-            // probabilities times value norms, transposed through shared memory (rows >= 4 of
-            // the tile stay zero in PACK4 mode)
-            if (writes_p) {
+            // probabilities times value norms, split into fp16 hi + lo and transposed through shared
+            // memory.  PACK4: tile rows 0..3 carry the hi parts (written by t4 < 2) and rows 4..7 the
+            // lo parts of the same rows (written by t4 >= 2, which hold the same row values).
+            {
                 const float pa = va ? vna : 0.f, pb = vb ? vnb : 0.f;
-                ptile[ra * 16 + gid] = __half_as_ushort(__float2half_rn(p0 * pa));
-                ptile[(ra + 1) * 16 + gid] = __half_as_ushort(__float2half_rn(p1 * pa));
-                ptile[ra * 16 + gid + 8] = __half_as_ushort(__float2half_rn(p2 * pb));
-                ptile[(ra + 1) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(p3 * pb));
+                const float w[4] = {p0 * pa, p1 * pa, p2 * pb, p3 * pb};
+                uint16_t hb[4], lb[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __half h = __float2half_rn(w[e]);
+                    hb[e] = __half_as_ushort(h);
+                    lb[e] = __half_as_ushort(__float2half_rn(w[e] - __half2float(h)));
+                }
+                if constexpr (PACK4) {
+                    const int row = t4 < 2 ? ra : ra + 4;
+                    const uint16_t *src = t4 < 2 ? hb : lb;
+                    ptile[row * 16 + gid] = src[0];
+                    ptile[(row + 1) * 16 + gid] = src[1];
+                    ptile[row * 16 + gid + 8] = src[2];
+                    ptile[(row + 1) * 16 + gid + 8] = src[3];
+                } else {
+                    ptile[ra * 16 + gid] = hb[0];
+                    ptile[(ra + 1) * 16 + gid] = hb[1];
+                    ptile[ra * 16 + gid + 8] = hb[2];
+                    ptile[(ra + 1) * 16 + gid + 8] = hb[3];
+                    ptile_lo[ra * 16 + gid] = lb[0];
+                    ptile_lo[(ra + 1) * 16 + gid] = lb[1];
+                    ptile_lo[ra * 16 + gid + 8] = lb[2];
+                    ptile_lo[(ra + 1) * 16 + gid + 8] = lb[3];
+                }
             }
             __syncwarp();
             const uint32_t bp0 = *(const uint32_t *)(ptile + gid * 16 + 2 * t4);
             const uint32_t bp1 = *(const uint32_t *)(ptile + gid * 16 + 2 * t4 + 8);
+            uint32_t bl0 = 0, bl1 = 0;
+            if constexpr (!PACK4) {
+                bl0 = *(const uint32_t *)(ptile_lo + gid * 16 + 2 * t4);
+                bl1 = *(const uint32_t *)(ptile_lo + gid * 16 + 2 * t4 + 8);
+            }
             __syncwarp();
             // ---------------- values: A = Vhat^T (coordinates x tokens), pairs along tokens
             {
-                uint32_t v0[VWPT], v1[VWPT], v8[VWPT], v9[VWPT];
                 const int tk = ob + 2 * t4;
-                load_words<VWPT>(svc + tk * VWPT, v0);
-                load_words<VWPT>(svc + (tk + 1) * VWPT, v1);
-                load_words<VWPT>(svc + (tk + 8) * VWPT, v8);
-                load_words<VWPT>(svc + (tk + 9) * VWPT, v9);
-#pragma unroll
-                for (int g = 0; g < G32; ++g) {
+                // pair index of (token 2i, token 2i+1) for one coordinate: 2*VB bits; for VB <= 3
+                // the byte holds index*4 (the table offset), for VB == 4 the index itself
+                constexpr int VSH = (VB <= 3) ? 2 : 0;
+                auto value_group = [&](int g, const uint32_t *w0, const uint32_t *w1, const uint32_t *w8,
+                                       const uint32_t *w9) {
                     uint32_t z0w = 0, z1w = 0, z8w = 0, z9w = 0;
 #pragma unroll
                     for (int p = 0; p < VB; ++p) {
-                        z0w |= ((v0[g * VB + p] >> gid) & 0x01010101u) << p;
-                        z1w |= ((v1[g * VB + p] >> gid) & 0x01010101u) << p;
-                        z8w |= ((v8[g * VB + p] >> gid) & 0x01010101u) << p;
-                        z9w |= ((v9[g * VB + p] >> gid) & 0x01010101u) << p;
+                        z0w |= ((w0[p] >> gid) & 0x01010101u) << p;
+                        z1w |= ((w1[p] >> gid) & 0x01010101u) << p;
+                        z8w |= ((w8[p] >> gid) & 0x01010101u) << p;
+                        z9w |= ((w9[p] >> gid) & 0x01010101u) << p;
                     }
-                    const uint32_t zz01 = (z0w << 2) | (z1w << (VB + 2));
-                    const uint32_t zz89 = (z8w << 2) | (z9w << (VB + 2));
+                    const uint32_t zz01 = (z0w << VSH) | (z1w << (VB + VSH));
+                    const uint32_t zz89 = (z8w << VSH) | (z9w << (VB + VSH));
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
+                        uint32_t o4[4] = {(zz01 >> (16 * h)) & 0xFFu, (zz01 >> (16 * h + 8)) & 0xFFu,
+                                          (zz89 >> (16 * h)) & 0xFFu, (zz89 >> (16 * h + 8)) & 0xFFu};
                         uint32_t a[4];
-                        a[0] = lut32(vlut, (zz01 >> (16 * h)) & 0xFFu);
-                        a[1] = lut32(vlut, (zz01 >> (16 * h + 8)) & 0xFFu);
-                        a[2] = lut32(vlut, (zz89 >> (16 * h)) & 0xFFu);
-                        a[3] = lut32(vlut, (zz89 >> (16 * h + 8)) & 0xFFu);
+                        uint32_t al[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint2 e = lut64(vlut, VSH ? (o4[u] << 1) : (o4[u] << 3));
+                            a[u] = e.x;
+                            al[u] = e.y;
+                        }
                         mma16816(oacc[2 * g + h], a, bp0, bp1);
+                        mma16816(oacc[2 * g + h], al, bp0, bp1);
+                        if constexpr (!PACK4) mma16816(oacc[2 * g + h], a, bl0, bl1);
+                    }
+                };
+                if constexpr (VB <= 3) {
+                    uint32_t v0[VWPT], v1[VWPT], v8[VWPT], v9[VWPT];
+                    load_words<VWPT>(svc + tk * VWPT, v0);
+                    load_words<VWPT>(svc + (tk + 1) * VWPT, v1);
+                    load_words<VWPT>(svc + (tk + 8) * VWPT, v8);
+                    load_words<VWPT>(svc + (tk + 9) * VWPT, v9);
+#pragma unroll
+                    for (int g = 0; g < G32; ++g) value_group(g, v0 + g * VB, v1 + g * VB, v8 + g * VB, v9 + g * VB);
+                } else {
+#pragma unroll
+                    for (int g = 0; g < G32; ++g) {
+                        uint32_t v0[VB], v1[VB], v8[VB], v9[VB];
+                        load_words<VB>(svc + tk * VWPT + g * VB, v0);
+                        load_words<VB>(svc + (tk + 1) * VWPT + g * VB, v1);
+                        load_words<VB>(svc + (tk + 8) * VWPT + g * VB, v8);
+                        load_words<VB>(svc + (tk + 9) * VWPT + g * VB, v9);
+                        value_group(g, v0, v1, v8, v9);
                     }
                 }
             }
@@ -472,6 +525,13 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     for (int o = 4; o < 32; o <<= 1) {
         l0 += __shfl_xor_sync(kFull, l0, o);
         l1 += __shfl_xor_sync(kFull, l1, o);
+    }
+    if constexpr (PACK4) {
+        // columns 4..7 (threads t4 >= 2) hold the lo-part products of rows 0..3
+#pragma unroll
+        for (int c = 0; c < KSTEP; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oacc[c][e] += __shfl_xor_sync(kFull, oacc[c][e], 2);
     }
     __syncthreads();
     float *comb = (float *)(smem + L.stage);  // [warp][row][D + 2]
@@ -546,6 +606,7 @@ cudaError_t launch_dm_bits(const Prepared &P, const ScoreProblem &sp, const floa
     if constexpr (ATTEND) {
         if (kb == 1 && vb == 2) return launch_dm_pack<D, 1, 2, true>(P, sp, qprep, scale, out, splits, s);
         if (kb == 2 && vb == 3) return launch_dm_pack<D, 2, 3, true>(P, sp, qprep, scale, out, splits, s);
+        if (kb == 3 && vb == 4) return launch_dm_pack<D, 3, 4, true>(P, sp, qprep, scale, out, splits, s);
     } else {
         // scores only: the value bit width is irrelevant
         if (kb == 1) return launch_dm_pack<D, 1, 1, false>(P, sp, qprep, scale, out, splits, s);
@@ -563,7 +624,7 @@ bool decode_mma_supported(const Prepared &P, const ScoreProblem &sp, bool attend
     const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
     if (!attend && rows > 64) return false;
     const int kb = P.kbeta, vb = P.vbeta;
-    if (attend) return (kb == 1 && vb == 2) || (kb == 2 && vb == 3);
+    if (attend) return vb == kb + 1 && kb >= 1 && kb <= 3;
     return kb >= 1 && kb <= 3;
 }
 
