@@ -460,9 +460,14 @@ def run_workload(args):
         tv = torch.empty((1, 1, Nq, k), dtype=torch.float32, device="cuda")
         scr = torch.empty(tq.tq_scores_scratch_bytes(p, 1, 1, 1, Nq, N, k), dtype=torch.uint8, device="cuda")
         ms = timed(lambda: tq.tq_scores(p, Qv, keys, 1, N, want_scores=False, topk=k, topk_idx=ti, topk_val=tv,
-                                        scratch=scr), steps=1, warmup=1)
+                                        scratch=scr), steps=5, warmup=3)
         r = rec("scores_top10", ms, N * Nq, "query_key_pairs", N * kb)
         r["tflops_equiv"] = 2.0 * Nq * N * (d + m) / (ms * 1e-3) / 1e12
+        # tensor-core work actually issued: fp16 hi/lo split products, 3 per centroid column and
+        # 2 per sign column, on 128-padded tiles
+        pad = lambda x: (x + 127) // 128 * 128
+        r["tflops_mma"] = 2.0 * pad(Nq) * pad(N) * (3 * d + 2 * m) / (ms * 1e-3) / 1e12
+        r["frac_tensor"] = r["tflops_mma"] / pk["bf16_tflops"] if pk.get("bf16_tflops") else None
         out.append(r)
         name = "vector search: 1M x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
     else:

@@ -163,8 +163,10 @@ size_t tq_scores_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int N
     Prepared P = prepared_view(p);
     ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                    nullptr);
+    const ScoresPlan plan = plan_scores(P, sp, topk);
     size_t bytes = qprep_bytes(P, sp);
-    if (topk > 0) bytes += topk_scratch_bytes(P, sp, topk);
+    if (plan.search) bytes += search_scratch_bytes(P, sp, plan.fused_topk ? topk : 0);
+    if (topk > 0 && !plan.fused_topk) bytes += topk_scratch_bytes(P, sp, topk);
     return bytes;
 }
 
@@ -172,7 +174,6 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
                     const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
                     const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx, float *topk_val,
                     void *scratch, size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
-    (void)dev_status;
     tq_status st = check_params(p, true);
     if (st != TQ_OK) return st;
     st = check_problem(p, B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm);
@@ -187,16 +188,26 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     Prepared P = prepared_view(p);
     ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm, nullptr, nullptr);
     cudaStream_t s = (cudaStream_t)stream;
-    float *qprep = (float *)scratch;
+    const ScoresPlan plan = plan_scores(P, sp, topk);
+    char *cur = (char *)scratch;
+    float *qprep = (float *)cur;
+    cur += qprep_bytes(P, sp);
+    void *search_scratch = cur;
+    if (plan.search) cur += search_scratch_bytes(P, sp, plan.fused_topk ? topk : 0);
     float *sbuf = scores;
-    if (!sbuf) sbuf = (float *)((char *)scratch + qprep_bytes(P, sp));
+    if (!sbuf && !plan.fused_topk) sbuf = (float *)cur;
     cudaError_t e = launch_qprep(P, sp, qprep, s);
-    if (e == cudaSuccess) {
-        if (decode_mma_supported(P, sp, false))
-            e = launch_decode_mma(P, sp, qprep, 1.0f, sbuf, decode_mma_splits(sp), false, s);
-        else
-            e = launch_scores(P, sp, qprep, sbuf, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (plan.fused_topk) {
+        e = launch_search(P, sp, qprep, search_scratch, scores, topk, topk_idx, topk_val, dev_status, s);
+        return from_cuda(e);
     }
+    if (plan.search)
+        e = launch_search(P, sp, qprep, search_scratch, sbuf, 0, nullptr, nullptr, dev_status, s);
+    else if (plan.mma)
+        e = launch_decode_mma(P, sp, qprep, 1.0f, sbuf, decode_mma_splits(sp), false, s);
+    else
+        e = launch_scores(P, sp, qprep, sbuf, s);
     if (e == cudaSuccess && topk > 0) e = launch_topk(sp, sbuf, topk, topk_idx, topk_val, s);
     return from_cuda(e);
 }

@@ -158,6 +158,28 @@ inline AttendPlan plan_attend(const Prepared &P, const ScoreProblem &sp) {
 }
 size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
 
+// Many query rows per (batch, KV head): tensor-core scores with an optional fused top-k.
+bool search_tc_supported(const Prepared &P, const ScoreProblem &sp, int topk);
+size_t search_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
+cudaError_t launch_search(const Prepared &P, const ScoreProblem &sp, const float *qprep, void *scratch,
+                          float *scores, int topk, int32_t *topk_idx, float *topk_val, int32_t *dev_status,
+                          cudaStream_t s);
+
+// Which kernels tq_scores runs: the tensor-core search (top-k fused when short enough), the
+// register-MMA decode kernel (few rows), or the plain kernel; a separate top-k pass otherwise.
+struct ScoresPlan {
+    bool search;      // launch_search
+    bool fused_topk;  // the search keeps the top-k itself
+    bool mma;         // launch_decode_mma in scores mode
+};
+inline ScoresPlan plan_scores(const Prepared &P, const ScoreProblem &sp, int topk) {
+    ScoresPlan a;
+    a.fused_topk = topk > 0 && search_tc_supported(P, sp, topk);
+    a.search = a.fused_topk || search_tc_supported(P, sp, 0);
+    a.mma = !a.search && decode_mma_supported(P, sp, false);
+    return a;
+}
+
 cudaError_t launch_qprep(const Prepared &P, const ScoreProblem &sp, float *qprep, cudaStream_t s);
 cudaError_t launch_scores(const Prepared &P, const ScoreProblem &sp, const float *qprep,
                           float *scores, cudaStream_t s);

@@ -171,7 +171,14 @@ def test_scratch_size_helpers(lib):
     p = _Params(128, 3, 64, 0x10000, 0x10000, 0x10000, ws)
     a = L.tq_attend_scratch_bytes(ctypes.byref(p), 32, 32, 8, 1, 32768)
     assert a >= 32 * 32 * (128 + 64) * 4
+    # few rows: a top-k pass over a full score buffer in scratch
+    f0 = L.tq_scores_scratch_bytes(ctypes.byref(p), 1, 1, 1, 16, 1000, 0)
+    f1 = L.tq_scores_scratch_bytes(ctypes.byref(p), 1, 1, 1, 16, 1000, 10)
+    assert f1 >= f0 + 16 * 1000 * 4
+    # many rows: a short top-k is fused (per-CTA lists only), a long one needs the score buffer
     s0 = L.tq_scores_scratch_bytes(ctypes.byref(p), 1, 1, 1, 1024, 1000, 0)
     s1 = L.tq_scores_scratch_bytes(ctypes.byref(p), 1, 1, 1, 1024, 1000, 10)
-    assert s1 >= s0 + 1024 * 1000 * 4
+    s2 = L.tq_scores_scratch_bytes(ctypes.byref(p), 1, 1, 1, 1024, 1000, 64)
+    assert s0 < s1 < s0 + 1024 * 1000 * 4
+    assert s2 >= s0 + 1024 * 1000 * 4
     assert L.tq_attend_scratch_bytes(ctypes.byref(p), 1, 3, 2, 1, 10) == 0

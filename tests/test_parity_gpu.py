@@ -176,6 +176,80 @@ def test_scores_topk_exact_ties(tq):
     np.testing.assert_array_equal(ti[0, 0, 0].cpu().numpy(), np.arange(100 * best, 100 * best + 10))
 
 
+@pytest.mark.parametrize("cfg", [
+    dict(d=128, m=64, bits=3, B=1, Hkv=1, G=1, Nq=200, T=1000),   # two row blocks, ragged keys
+    dict(d=64, m=64, bits=2, B=2, Hkv=2, G=3, Nq=30, T=300),      # GQA slices, 1-bit keys
+    dict(d=256, m=128, bits=4, B=1, Hkv=1, G=1, Nq=129, T=129),   # one row past a block
+    # vector-search width with the search workload's unit keys and queries: the 1e-4 absolute
+    # bound presumes that scale (with |q| |k| ~ d = 1024, plain fp32 summation alone already
+    # rounds near-zero scores by more than 1e-4)
+    dict(d=1024, m=512, bits=4, B=1, Hkv=1, G=1, Nq=130, T=300, unit=True),
+    dict(d=128, m=128, bits=3, B=1, Hkv=1, G=1, Nq=65, T=1),      # single key
+])
+def test_search_scores_and_topk(tq, cfg):
+    """Many query rows per KV head (the tensor-core path): full scores, and the top-k both fused
+    (k <= 16) and as a separate pass (k > 16), against the oracle."""
+    import torch
+    c = cfg
+    seed = 300 + c["d"] + c["T"]
+    if c.get("unit"):
+        R = synth.rotation(c["d"], seed)
+        S = synth.gaussian(c["m"], c["d"], seed + 1)
+        K = synth.unit_rows(c["B"] * c["Hkv"] * c["T"], c["d"], seed + 2)
+        k = oracle.compress(K, R, S, c["bits"], is_key=True)
+    else:
+        R, S, k, _ = _oracle_cache(seed, c["d"], c["m"], c["bits"], c["B"], c["Hkv"], c["T"], f16=False)
+    Hq = c["Hkv"] * c["G"]
+    rows = c["B"] * Hq * c["Nq"]
+    q = (synth.unit_rows(rows, c["d"], 9) if c.get("unit") else synth.gaussian(rows, c["d"], 9))
+    q = q.reshape(c["B"], Hq, c["Nq"], c["d"])
+    ora = oracle.scores(q, R, S, c["bits"], c["B"], Hq, c["Hkv"], c["Nq"], c["T"],
+                        k["codes"], k["signs"], k["norm"], k["rnorm"])
+    p = _params(tq, R, S, c["bits"], c["m"])
+    qd = torch.from_numpy(q).cuda()
+    s, _, _ = tq.tq_scores(p, qd, _to_dev(k), c["Hkv"], c["T"])
+    torch.cuda.synchronize()
+    check_close(s, ora, "scores")
+    for k_ in (1, 10, 16, 20):
+        if k_ > c["T"]:
+            continue
+        for want_scores in (False, True):
+            s2, ti, tv = tq.tq_scores(p, qd, _to_dev(k), c["Hkv"], c["T"], want_scores=want_scores, topk=k_)
+            torch.cuda.synchronize()
+            ti, tv = ti.cpu().numpy(), tv.cpu().numpy()
+            for b in range(c["B"]):
+                for h in range(Hq):
+                    for r in range(0, c["Nq"], 7):
+                        check_topk(ti[b, h, r], tv[b, h, r], ora[b, h, r], k_, f"k={k_} row {b},{h},{r}")
+            if want_scores:
+                # the top-k is exactly the k best of the returned scores
+                sc = s2.cpu().numpy()
+                for r in range(0, c["Nq"], 11):
+                    row = sc[0, 0, r].astype(np.float64)
+                    order = np.lexsort((np.arange(c["T"]), -row))[:k_]
+                    np.testing.assert_array_equal(ti[0, 0, r], order)
+
+
+def test_search_topk_exact_ties(tq):
+    # identical keys, many query rows: ties resolve to the smaller token index across CTAs too
+    import torch
+    d, m, bits, T, Nq = 64, 64, 3, 4000, 100
+    R = synth.rotation(d, 11)
+    S = synth.gaussian(m, d, 12)
+    K = np.repeat(synth.gaussian(8, d, 13), 500, axis=0)
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    q = synth.gaussian(Nq, d, 14).reshape(1, 1, Nq, d)
+    p = _params(tq, R, S, bits, m)
+    _, ti, _ = tq.tq_scores(p, torch.from_numpy(q).cuda(), _to_dev(k), 1, T, want_scores=False, topk=16)
+    ora = oracle.scores(q, R, S, bits, 1, 1, 1, Nq, T, k["codes"], k["signs"], k["norm"], k["rnorm"])[0, 0]
+    for r in range(Nq):
+        vals = ora[r, ::500]
+        best = int(np.argmax(vals))
+        if np.sort(vals)[-2] > vals[best] - 1e-3 * abs(vals[best]) - 1e-4:
+            continue  # two groups too close to call
+        np.testing.assert_array_equal(ti[0, 0, r].cpu().numpy(), np.arange(500 * best, 500 * best + 16))
+
+
 # -------------------------------------------------------------------- attend
 
 @pytest.mark.parametrize("cfg", [
