@@ -31,38 +31,66 @@ inline int rows_per_pass(int d, int m, int cap_regs) {
 
 // ------------------------------------------------------------------ query prep
 
-constexpr int kQprepRows = 8;
+constexpr int kQpR = 64;   // query rows per block tile
+constexpr int kQpC = 64;   // output coordinates per block tile
+constexpr int kQpK = 16;   // input coordinates per shared-memory step
 
-// q_rot = R q and sq = S q for kQprepRows query rows per block: each thread owns one output
-// coordinate and carries one accumulator per row (the R^T / S^T row it reads is shared).
-__global__ void qprep_kernel(Prepared P, const float *__restrict__ q, int64_t rows,
-                             float *__restrict__ out) {
-    extern __shared__ float qs[];  // [kQprepRows][d]
-    const int d = P.d, m = P.m;
-    for (int64_t r0 = (int64_t)blockIdx.x * kQprepRows; r0 < rows; r0 += (int64_t)gridDim.x * kQprepRows) {
-        const int nr = (int)min((int64_t)kQprepRows, rows - r0);
-        for (int e = threadIdx.x; e < kQprepRows * d; e += blockDim.x) {
-            const int r = e / d, j = e % d;
-            qs[e] = r < nr ? q[(r0 + r) * d + j] : 0.f;
-        }
-        __syncthreads();
-        for (int i = threadIdx.x; i < d + m; i += blockDim.x) {
-            const bool rot = i < d;
-            const float *mat = rot ? P.RT + i : P.ST + (i - d);
-            const int ld = rot ? d : m;
-            float acc[kQprepRows];
+// q_rot = R q and sq = S q as one fp32 GEMM, out[r][i] = sum_j q[r][j] W[j][i] with
+// W = [R^T | S^T]: 64 x 64 output tiles, 4 x 4 per thread, operands staged in shared memory.
+// Every output is accumulated by fmaf in ascending j, so the result does not depend on the
+// tiling.
+__global__ void __launch_bounds__(256) qprep_kernel(Prepared P, const float *__restrict__ q, int64_t rows,
+                                                    float *__restrict__ out) {
+    __shared__ float qs[kQpK][kQpR + 4];  // q tile, transposed
+    __shared__ __align__(16) float ws[kQpK][kQpC];
+    const int d = P.d, m = P.m, n = d + m;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int c0 = blockIdx.x * kQpC;
+    for (int64_t r0 = (int64_t)blockIdx.y * kQpR; r0 < rows; r0 += (int64_t)gridDim.y * kQpR) {
+        float acc[4][4];
 #pragma unroll
-            for (int r = 0; r < kQprepRows; ++r) acc[r] = 0.f;
-            for (int j = 0; j < d; ++j) {
-                const float w = mat[(int64_t)j * ld];
+        for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int r = 0; r < kQprepRows; ++r) acc[r] = fmaf(w, qs[r * d + j], acc[r]);
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int k0 = 0; k0 < d; k0 += kQpK) {
+            for (int e = tid; e < kQpR * kQpK; e += 256) {
+                const int r = e / kQpK, k = e % kQpK;
+                qs[k][r] = r0 + r < rows ? q[(r0 + r) * d + k0 + k] : 0.f;
             }
+            for (int e = tid; e < kQpK * kQpC; e += 256) {
+                const int k = e / kQpC, c = e % kQpC, i = c0 + c, j = k0 + k;
+                float w = 0.f;
+                if (i < d) w = P.RT[(int64_t)j * d + i];
+                else if (i < n) w = P.ST[(int64_t)j * m + (i - d)];
+                ws[k][c] = w;
+            }
+            __syncthreads();
 #pragma unroll
-            for (int r = 0; r < kQprepRows; ++r)
-                if (r < nr) out[(r0 + r) * (d + m) + i] = acc[r];
+            for (int k = 0; k < kQpK; ++k) {
+                float a[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) a[t] = qs[k][ty * 4 + t];
+                const float4 b = *(const float4 *)&ws[k][tx * 4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    acc[t][0] = fmaf(b.x, a[t], acc[t][0]);
+                    acc[t][1] = fmaf(b.y, a[t], acc[t][1]);
+                    acc[t][2] = fmaf(b.z, a[t], acc[t][2]);
+                    acc[t][3] = fmaf(b.w, a[t], acc[t][3]);
+                }
+            }
+            __syncthreads();
         }
-        __syncthreads();
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int64_t r = r0 + ty * 4 + t;
+            if (r >= rows) continue;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = c0 + tx * 4 + u;
+                if (i < n) out[r * n + i] = acc[t][u];
+            }
+        }
     }
 }
 
@@ -410,11 +438,9 @@ size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk) {
 
 cudaError_t launch_qprep(const Prepared &P, const ScoreProblem &sp, float *qprep, cudaStream_t s) {
     const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
-    const int64_t groups = (rows + kQprepRows - 1) / kQprepRows;
-    int blocks = (int)(groups < 148 * 8 ? groups : 148 * 8);
-    const size_t smem = sizeof(float) * kQprepRows * P.d;
-    cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    qprep_kernel<<<blocks, 128, smem, s>>>(P, sp.q, rows, qprep);
+    const int64_t rtiles = (rows + kQpR - 1) / kQpR;
+    dim3 grid((unsigned)((P.d + P.m + kQpC - 1) / kQpC), (unsigned)(rtiles < 65535 ? rtiles : 65535));
+    qprep_kernel<<<grid, 256, 0, s>>>(P, sp.q, rows, qprep);
     return cudaGetLastError();
 }
 
