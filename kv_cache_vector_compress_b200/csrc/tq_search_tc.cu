@@ -5,15 +5,16 @@
 // Python-implementasjonen?"; the score is the asymmetric estimator of "turboquant-pytorch",
 // nav.superapi.store, 核心 API):
 //   s[r, t] = ||k_t|| ( <q_rot_r, c[idx_t]> + rho_t sqrt(pi/2)/m <sq_r, 2 sign_t - 1> )
-// computed as two GEMMs per tile of 128 keys x 128 query rows, K streamed in 64-wide blocks:
-//   ACC1 = C (centroids, fp16 hi + lo) x Qrot^T (fp16 hi + lo)    three products per block
-//   ACC2 = Sgn (+-1, exact) x SQ^T (fp16 hi + lo)                  two products per block
-// Decoder warps write the keys' A tiles straight into the 128-byte-swizzled shared-memory layout
-// from the packed codes; the queries' B tiles (split and swizzled once per call) arrive by bulk
-// copy; tcgen05 accumulates into one of two TMEM slots while the epilogue turns the other slot
-// into scores, transposes them through shared memory and keeps each query row's running top-k.
-// A merge kernel combines the per-CTA lists.  Every operand product is exact in fp32 up to the
-// dropped lo x lo terms (relative 2^-22), so the result matches fp32 evaluation of the formula.
+// computed per tile of 128 keys x 128 query rows as one GEMM with K = d + m, streamed in
+// 64-wide blocks into a single fp32 accumulator:
+//   centroid blocks: C (fp16 hi + lo) x Qrot^T (fp16 hi + lo)          three products
+//   sign blocks:     (+-rho_t, exact in fp16) x (gamma SQ)^T (hi + lo)   two products
+// Decoder warps turn the packed codes of each key into its A rows and store them straight into
+// tensor memory (the MMA reads A from TMEM, so shared-memory bandwidth is left to the B tiles);
+// the queries' B tiles are split and swizzled once per call and arrive by bulk copy.  Two TMEM
+// accumulator slots let the epilogue of one tile overlap the MMAs of the next; it transposes the
+// scores through shared memory and keeps running per-row top-k lists, merged by a small kernel.
+// Every operand product is exact in fp32 up to the dropped lo x lo terms (relative 2^-22).
 #include <math.h>
 
 #include "tq_common.cuh"
@@ -26,46 +27,61 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kSTile = 128;                    // keys per tile (MMA M) and query rows per tile (MMA N)
-constexpr int kSThreads = 448;                 // 14 warps
-constexpr int kDecWarp0 = 2;                   // warps 2..9 decode key tiles
-constexpr int kEpiWarp0 = 10;                  // warps 10..13 epilogue
-constexpr int kSStages = 2;                    // shared-memory operand stages
-constexpr uint32_t kOpTile = kSTile * 128;     // one 128 x 64 fp16 operand tile (16 KB)
-constexpr uint32_t kStageBytes = 4 * kOpTile;  // A hi, A lo, B hi, B lo
-constexpr int kScStride = kSTile + 1;          // transposed score tile row stride (floats)
-constexpr int kSearchSms = 148;                // grid sizing (fixed so scratch sizes do not vary)
-constexpr int kMaxFusedTopk = 16;              // longest per-row list kept in shared memory
+constexpr int kSTile = 128;                  // keys per tile (MMA M) and query rows per tile (MMA N)
+constexpr int kDecGroups = 2;                // key-decoder groups of four warps, one K-block each in turn
+constexpr int kDecWarp0 = 2;                 // warps 2 .. 2 + 4 kDecGroups - 1: key decoders
+constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;  // four epilogue warps
+constexpr int kSThreads = 32 * (kEpiWarp0 + 4);
+constexpr int kSStages = 4;                  // operand stages (B in shared memory, A in TMEM)
+constexpr uint32_t kBTile = kSTile * 128;    // one 128 x 64 fp16 B tile (16 KB)
+constexpr uint32_t kStageBytes = 2 * kBTile; // B hi, B lo
+constexpr uint32_t kAccCols = 128;           // accumulator columns per slot
+constexpr uint32_t kACol0 = 2 * kAccCols;    // first TMEM column of the A stages
+constexpr uint32_t kAStageCols = 64;         // A hi (32 columns) | A lo (32 columns) per stage
+constexpr int kScRows = 64;                  // query rows transposed at a time
+constexpr int kScStride = kSTile + 4;        // transposed score row stride (floats, 16-byte rows)
+constexpr int kSearchSms = 148;              // grid sizing (fixed so scratch sizes do not vary)
+constexpr int kMaxFusedTopk = 16;            // longest per-row list kept in shared memory
+
+constexpr int kQCap = 24;                    // per-row candidate queue entries per tile
 
 struct SearchSmem {
-    uint32_t stage, sc, lv, li, rowoff, klut, bars, misc, total;
+    uint32_t stage, sc, lv, li, qv, qi, thr, qcnt, klut, rowoff, bars, misc, total;
 };
 
-__host__ __device__ inline SearchSmem search_smem_layout(int K) {
+__host__ __device__ inline SearchSmem search_smem_layout(int K, int KB) {
     SearchSmem L;
     uint32_t o = 0;
     L.stage = o;
     o += kSStages * kStageBytes;
-    L.sc = o;
-    o += kSTile * kScStride * 4;
-    L.lv = o;
+    L.sc = o;  // transposed scores of 64 query rows (overflow path)
+    o += kScRows * kScStride * 4;
+    L.lv = o;  // per-row top-k lists, K entries each, padded with (-inf, INT32_MAX)
     o += kSTile * (K > 0 ? K : 1) * 4;
     L.li = o;
     o += kSTile * (K > 0 ? K : 1) * 4;
+    L.qv = o;  // per-row candidate queues of the current tile
+    o += kSTile * kQCap * 4;
+    L.qi = o;
+    o += kSTile * kQCap * 4;
+    L.thr = o;  // per-row admission threshold (the k-th best so far, -inf until k are held)
+    o += kSTile * 4;
+    L.qcnt = o;
+    o += kSTile * 4;
     o = (o + 15) & ~15u;
+    L.klut = o;
+    o += (1u << (2 * KB)) * 32 * 8;
     L.rowoff = o;
     o += kSTile * 8;
-    L.klut = o;
-    o += 64 * 8;
     L.bars = o;
-    o += 16 * 8;
+    o += 32 * 8;
     L.misc = o;
     o += 64;
     L.total = o;
     return L;
 }
 
-enum SBar { kBFull = 0, kAFull = 2, kSEmpty = 4, kAccFull = 6, kAccEmpty = 8 };
+enum SBar { kBFull = 0, kAFull = 4, kSEmpty = 8, kAccFull = 12, kAccEmpty = 14 };
 
 struct SearchGeom {
     int d, m;
@@ -107,34 +123,34 @@ __device__ __forceinline__ uint32_t pack_h2s(float lo, float hi) {
     return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
 }
 __device__ __forceinline__ float hi16(float x) { return __half2float(__float2half_rn(x)); }
-// Exponent e with maxabs * 2^e in [512, 1024): the fp16 operands stay far from overflow and
-// their lo halves far from the subnormal range.
+// Exponent e with maxabs * 2^e in [512, 1024): fp16 operands far from overflow, and their lo
+// halves far from the subnormal range.
 __device__ __forceinline__ int pow2_exp(float maxabs) {
     if (!(maxabs > 0.f) || !isfinite(maxabs)) return 0;
     int e;
     frexpf(maxabs, &e);
     return 10 - e;
 }
+__device__ __forceinline__ float search_gamma(int m) { return sqrtf(1.5707963267948966f) / (float)m; }
 
 // ------------------------------------------------------------------ query operands
 
-// Per unit (slice, block of 128 query rows): one scale exponent for the rotated-query columns and
-// one for the projected-query columns, and the B operand tiles -- fp16 hi | lo of the scaled
-// values -- in the 128-byte-swizzled K-major layout, K-block by K-block.
-__global__ void search_prep_kernel(ScoreProblem sp, SearchGeom g, const float *__restrict__ qprep,
-                                   uint8_t *__restrict__ qsw, int *__restrict__ uexp) {
-    __shared__ float red[2][32];
-    __shared__ int ex[2];
-    const int unit = blockIdx.x;
-    const int d = g.d, m = g.m, stride = d + m;
+// Per unit (slice, block of 128 query rows): max |q_rot| and max |gamma sq| over its rows, as
+// float bits (non-negative floats order like their bit patterns); umax starts at zero.
+__global__ void search_max_kernel(ScoreProblem sp, SearchGeom g, const float *__restrict__ qprep,
+                                  unsigned *__restrict__ umax) {
+    __shared__ float red[2][8];
+    const int unit = blockIdx.x, rows_per = kSTile / gridDim.y;
+    const int d = g.d, stride = g.d + g.m;
+    const float gamma = search_gamma(g.m);
     float qm = 0.f, sm = 0.f;
-    for (int e = threadIdx.x; e < kSTile * stride; e += blockDim.x) {
-        const int r = e / stride, col = e % stride;
+    for (int e = threadIdx.x; e < rows_per * stride; e += blockDim.x) {
+        const int r = blockIdx.y * rows_per + e / stride, col = e % stride;
         const int64_t qr = search_qrow(sp, g, unit, r);
         if (qr < 0) continue;
-        const float v = fabsf(qprep[qr * stride + col]);
-        if (col < d) qm = fmaxf(qm, v);
-        else sm = fmaxf(sm, v);
+        const float v = qprep[qr * stride + col];
+        if (col < d) qm = fmaxf(qm, fabsf(v));
+        else sm = fmaxf(sm, fabsf(gamma * v));
     }
     qm = warp_max(qm);
     sm = warp_max(sm);
@@ -147,28 +163,59 @@ __global__ void search_prep_kernel(ScoreProblem sp, SearchGeom g, const float *_
     if (threadIdx.x < 2) {
         float mx = 0.f;
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, red[threadIdx.x][w]);
-        ex[threadIdx.x] = pow2_exp(mx);
-        uexp[unit * 2 + threadIdx.x] = ex[threadIdx.x];
+        atomicMax(&umax[unit * 2 + threadIdx.x], __float_as_uint(mx));
     }
-    __syncthreads();
-    const float s0 = ldexpf(1.f, ex[0]), s1 = ldexpf(1.f, ex[1]);
-    uint8_t *base = qsw + (size_t)unit * g.nkb * 2 * kOpTile;
-    for (int e = threadIdx.x; e < kSTile * stride; e += blockDim.x) {
-        const int r = e / stride, col = e % stride;
+}
+
+// Key-side centroid exponent: the codebook's largest |centroid| scaled into [512, 1024).
+__device__ __forceinline__ int centroid_exp(const Prepared &P) {
+    float kmax = 0.f;
+    for (int k = 0; k < (1 << P.kbeta); ++k) kmax = fmaxf(kmax, fabsf(P.cb->kc[k]));
+    return pow2_exp(kmax);
+}
+
+// One B tile (unit, K-block) per block: fp16 hi | lo of q_rot * 2^eq (centroid blocks) or of
+// gamma sq * 2^eB (sign blocks), in the 128-byte-swizzled K-major layout.  The exponents make
+// both parts of the accumulator carry the same scale 2^E: E = eq + ek for centroids (ek on the
+// key side) and E = eB + eA for signs, where the key side holds +-rho * 2^eA (exact in fp16
+// for eA in [-8, 14]).  E is lowered, if need be, so that eA <= 14 without pushing any B value
+// above its [512, 1024) target.  uexp[unit] = {E, eA}.
+__global__ void search_tiles_kernel(Prepared P, ScoreProblem sp, SearchGeom g, const float *__restrict__ qprep,
+                                    const unsigned *__restrict__ umax, uint8_t *__restrict__ qsw,
+                                    int *__restrict__ uexp) {
+    const int unit = blockIdx.x, kb = blockIdx.y;
+    const int d = g.d, stride = g.d + g.m, dkb = g.d / 64;
+    const int eq = pow2_exp(__uint_as_float(umax[unit * 2]));
+    const int ebn = pow2_exp(__uint_as_float(umax[unit * 2 + 1]));
+    const int ek = centroid_exp(P);
+    const int E = min(eq + ek, ebn + 14);
+    const int eA = max(-8, E - ebn);
+    if (kb == 0 && threadIdx.x == 0) {
+        uexp[unit * 2] = E;
+        uexp[unit * 2 + 1] = eA;
+    }
+    const bool sgn = kb >= dkb;
+    const float scale = sgn ? search_gamma(g.m) * ldexpf(1.f, E - eA) : ldexpf(1.f, E - ek);
+    const int col0 = sgn ? d + (kb - dkb) * 64 : kb * 64;
+    uint8_t *hi = qsw + ((size_t)unit * g.nkb + kb) * kStageBytes;
+    uint8_t *lo = hi + kBTile;
+    for (int e = threadIdx.x; e < kSTile * 64; e += blockDim.x) {
+        const int r = e >> 6, kk = e & 63;
         const int64_t qr = search_qrow(sp, g, unit, r);
-        const bool sgn = col >= d;
-        const float v = qr >= 0 ? qprep[qr * stride + col] * (sgn ? s1 : s0) : 0.f;
-        const int kb = sgn ? d / 64 + (col - d) / 64 : col / 64;
-        const int kk = (sgn ? col - d : col) & 63;
+        const float v = qr >= 0 ? qprep[qr * stride + col0 + kk] * scale : 0.f;
         const uint32_t off = (uint32_t)r * 128 + ((((uint32_t)kk >> 3) ^ (r & 7)) << 4) + (kk & 7) * 2;
         const __half h = __float2half_rn(v);
-        const __half lo = __float2half_rn(v - __half2float(h));
-        *(__half *)(base + (size_t)kb * 2 * kOpTile + off) = h;
-        *(__half *)(base + (size_t)kb * 2 * kOpTile + kOpTile + off) = lo;
+        *(__half *)(hi + off) = h;
+        *(__half *)(lo + off) = __float2half_rn(v - __half2float(h));
     }
 }
 
 // ------------------------------------------------------------------------ GEMM
+
+__device__ __forceinline__ bool search_better(float va, int32_t ia, float vb, int32_t ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
 
 template <int KB>
 __global__ void __launch_bounds__(kSThreads, 1)
@@ -179,30 +226,29 @@ __global__ void __launch_bounds__(kSThreads, 1)
     const int KWPT = KB * (g.d / 32);  // code words per key
     const int SWPT = g.m / 32;         // sign words per key
     const int NKB = g.nkb;
-    const SearchSmem L = search_smem_layout(K);
+    const SearchSmem L = search_smem_layout(K, KB);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t *bars = (uint64_t *)(sm + L.bars);
     float *sc = (float *)(sm + L.sc);
-    float *lv = (float *)(sm + L.lv);
-    int32_t *li = (int32_t *)(sm + L.li);
+    const uint2 *klut = (const uint2 *)(sm + L.klut);
     int64_t *rowoff = (int64_t *)(sm + L.rowoff);
-    uint2 *klut = (uint2 *)(sm + L.klut);
     uint32_t *tmem_s = (uint32_t *)(sm + L.misc);
     volatile int *abort_s = (volatile int *)(sm + L.misc + 4);
-    int *kexp_s = (int *)(sm + L.misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int unit = blockIdx.x / g.kc, cidx = blockIdx.x % g.kc;
     const int sl = unit / g.nrb;
     const int my_tiles = (int)((g.nkt - cidx + g.kc - 1) / g.kc);
+    const int total = my_tiles * NKB;
     const int64_t rec_base = (int64_t)sl * sp.T;
+    const int E = uexp[unit * 2], eA = uexp[unit * 2 + 1];
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSStages; ++s) {
             mbar_init(&bars[kBFull + s], 1);
-            mbar_init(&bars[kAFull + s], 8);
+            mbar_init(&bars[kAFull + s], 4);
             mbar_init(&bars[kSEmpty + s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -210,32 +256,36 @@ __global__ void __launch_bounds__(kSThreads, 1)
             mbar_init(&bars[kAccEmpty + s], 4);
         }
         *abort_s = 0;
-        float kmax = 0.f;
-        for (int k = 0; k < (1 << KB); ++k) kmax = fmaxf(kmax, fabsf(P.cb->kc[k]));
-        *kexp_s = pow2_exp(kmax);
         fence_mbar_init();
     }
-    __syncthreads();
     {
-        // centroid pair table (hi, lo) for two coordinates whose plane bits interleave in idx
-        const float ksc = ldexpf(1.f, *kexp_s);
-        for (int e = threadIdx.x; e < (1 << (2 * KB)); e += blockDim.x) {
+        // centroid pair table (hi pair, lo pair), one copy per lane so lookups never conflict:
+        // entry idx holds coordinates whose plane bits interleave in idx (even bits: first)
+        uint2 *lut = (uint2 *)(sm + L.klut);
+        const float ksc = ldexpf(1.f, centroid_exp(P));
+        for (int e = threadIdx.x; e < (32 << (2 * KB)); e += blockDim.x) {
+            const int idx = e >> 5;
             int i0 = 0, i1 = 0;
             for (int p = 0; p < KB; ++p) {
-                i0 |= ((e >> (2 * p)) & 1) << p;
-                i1 |= ((e >> (2 * p + 1)) & 1) << p;
+                i0 |= ((idx >> (2 * p)) & 1) << p;
+                i1 |= ((idx >> (2 * p + 1)) & 1) << p;
             }
             const float a0 = P.cb->kc[i0] * ksc, a1 = P.cb->kc[i1] * ksc;
-            klut[e] = make_uint2(pack_h2s(a0, a1), pack_h2s(a0 - hi16(a0), a1 - hi16(a1)));
+            lut[e] = make_uint2(pack_h2s(a0, a1), pack_h2s(a0 - hi16(a0), a1 - hi16(a1)));
         }
         for (int r = threadIdx.x; r < kSTile; r += blockDim.x) {
             const int64_t qr = search_qrow(sp, g, unit, r);
             rowoff[r] = qr < 0 ? -1 : qr * sp.T;
         }
         for (int e = threadIdx.x; e < kSTile * K; e += blockDim.x) {
-            lv[e] = -INFINITY;
-            li[e] = INT32_MAX;
+            ((float *)(sm + L.lv))[e] = -INFINITY;
+            ((int32_t *)(sm + L.li))[e] = INT32_MAX;
         }
+        for (int r = threadIdx.x; r < kSTile; r += blockDim.x) {
+            ((float *)(sm + L.thr))[r] = search_qrow(sp, g, unit, r) >= 0 ? -INFINITY : INFINITY;
+            ((int *)(sm + L.qcnt))[r] = 0;
+        }
+        if (threadIdx.x < 2) ((volatile int *)(sm + L.misc + 8))[threadIdx.x] = 0;  // queue overflow flags
     }
     if (warp == 0) {
         tmem_alloc(tmem_s, 512);
@@ -245,20 +295,18 @@ __global__ void __launch_bounds__(kSThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_s;
-    const uint8_t *qsw_u = qsw + (size_t)unit * NKB * 2 * kOpTile;
+    const uint8_t *qsw_u = qsw + (size_t)unit * NKB * kStageBytes;
 
     if (warp == 0) {
         // -------------------------------------------------------- query tiles (bulk copies)
         if (lane == 0) {
-            const int total = my_tiles * NKB;
             int issued = 0;
             for (int gk = 0; gk < total; ++gk) {
                 const int st = gk % kSStages;
                 if (gk >= kSStages && !mbar_wait(&bars[kSEmpty + st], ((gk / kSStages) - 1) & 1, abort_s)) break;
-                const int kbi = gk % NKB;
-                mbar_arrive_expect_tx(&bars[kBFull + st], 2 * kOpTile);
-                bulk_load(sm + L.stage + st * kStageBytes + 2 * kOpTile, qsw_u + (size_t)kbi * 2 * kOpTile,
-                          2 * kOpTile, &bars[kBFull + st]);
+                mbar_arrive_expect_tx(&bars[kBFull + st], kStageBytes);
+                bulk_load(sm + L.stage + st * kStageBytes, qsw_u + (size_t)(gk % NKB) * kStageBytes, kStageBytes,
+                          &bars[kBFull + st]);
                 issued = gk + 1;
             }
             // every copy must land before the CTA can exit (bounded waits)
@@ -267,7 +315,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
                 mbar_wait(&bars[kBFull + gk % kSStages], (gk / kSStages) & 1, (volatile int *)&dummy);
         }
     } else if (warp == 1) {
-        // -------------------------------------------------------- MMA issue
+        // -------------------------------------------------------- MMA issue (A from TMEM)
         if (lane == 0) {
             const uint32_t idesc = idesc_f16_f32(kSTile, kSTile);
             const uint32_t sbase = smem_u32(sm + L.stage);
@@ -276,33 +324,25 @@ __global__ void __launch_bounds__(kSThreads, 1)
                 const int slot = i & 1;
                 if (i >= 2 && !mbar_wait(&bars[kAccEmpty + slot], ((i >> 1) - 1) & 1, abort_s)) break;
                 tc_fence_after();
-                const uint32_t acc1 = tmem + slot * 256, acc2 = acc1 + kSTile;
+                const uint32_t acc = tmem + slot * kAccCols;
                 for (int kbi = 0; kbi < NKB; ++kbi) {
                     const int gk = i * NKB + kbi, st = gk % kSStages;
-                    if (!mbar_wait(&bars[kAFull + st], (gk / kSStages) & 1, abort_s) ||
-                        !mbar_wait(&bars[kBFull + st], (gk / kSStages) & 1, abort_s)) {
+                    const uint32_t ph = (gk / kSStages) & 1;
+                    if (!mbar_wait(&bars[kAFull + st], ph, abort_s) || !mbar_wait(&bars[kBFull + st], ph, abort_s)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_hi = sbase + st * kStageBytes, a_lo = a_hi + kOpTile;
-                    const uint32_t b_hi = a_hi + 2 * kOpTile, b_lo = a_hi + 3 * kOpTile;
-                    if (kbi < DKB) {
+                    const uint32_t a0 = tmem + kACol0 + st * kAStageCols;
+                    const uint32_t b_hi = sbase + st * kStageBytes, b_lo = b_hi + kBTile;
+                    const bool cen = kbi < DKB;
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t o = k * 32;
-                            mma_ss(acc1, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kbi | k) ? 1u : 0u);
-                            mma_ss(acc1, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
-                            mma_ss(acc1, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t o = k * 32;
-                            mma_ss(acc2, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc,
-                                   ((kbi - DKB) | k) ? 1u : 0u);
-                            mma_ss(acc2, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
-                        }
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t a_hi = a0 + 32 * (k >> 1) + 8 * (k & 1);
+                        const uint64_t dh = sdesc_sw128(b_hi + 32 * k), dl = sdesc_sw128(b_lo + 32 * k);
+                        mma_ts(acc, a_hi, dh, idesc, (kbi | k) ? 1u : 0u);
+                        mma_ts(acc, a_hi, dl, idesc, 1u);
+                        if (cen) mma_ts(acc, a_hi + 16, dh, idesc, 1u);
                     }
                     mma_commit(&bars[kSEmpty + st]);
                 }
@@ -310,147 +350,297 @@ __global__ void __launch_bounds__(kSThreads, 1)
             }
         }
     } else if (warp < kEpiWarp0) {
-        // -------------------------------------------------------- key tile decode
-        const int dt = threadIdx.x - kDecWarp0 * 32;  // 0..255
-        const int kr = dt & (kSTile - 1), half = dt >> 7;
-        const int total = my_tiles * NKB;
-        for (int gk = 0; gk < total; ++gk) {
-            const int st = gk % kSStages, kbi = gk % NKB, i = gk / NKB;
+        // -------------------------------------------------------- key decode into TMEM
+        // group g fills the K-block steps g, g + kDecGroups, ...; within a group the four warps
+        // cover the four TMEM lane quarters, one key per thread
+        const int grp = (warp - kDecWarp0) >> 2;
+        const int quarter = warp & 3;
+        const int kr = 32 * quarter + lane;
+        const uint32_t tq = tmem + ((uint32_t)(32 * quarter) << 16) + kACol0;
+        auto fetch = [&](int gk, uint2 (&u)[KB], uint32_t &rb, bool &valid) {
+            const int kbi = gk % NKB, i = gk / NKB;
             const int64_t t = (int64_t)(cidx + (int64_t)i * g.kc) * kSTile + kr;
-            const bool valid = t < sp.T;
-            // fetch the packed words before waiting for the stage to free up
-            uint32_t w[KB];
-            if (kbi < DKB) {
-                const uint32_t *src = sp.kcodes + (rec_base + t) * KWPT + (2 * kbi + half) * KB;
+            valid = t < sp.T;
 #pragma unroll
-                for (int p = 0; p < KB; ++p) w[p] = valid ? __ldg(src + p) : 0u;
+            for (int p = 0; p < KB; ++p) u[p] = make_uint2(0u, 0u);
+            rb = 0;
+            if (!valid) return;
+            const int64_t rec = rec_base + t;
+            if (kbi < DKB) {
+                const uint2 *src = (const uint2 *)(sp.kcodes + rec * KWPT + 2 * kbi * KB);
+#pragma unroll
+                for (int p = 0; p < KB; ++p) u[p] = __ldg(src + p);
             } else {
-                w[0] = valid ? __ldg(sp.ksigns + (rec_base + t) * SWPT + 2 * (kbi - DKB) + half) : 0u;
+                u[0] = __ldg((const uint2 *)(sp.ksigns + rec * SWPT + 2 * (kbi - DKB)));
+                rb = sp.krnorm[rec];
             }
+        };
+        uint2 cu[KB], nu[KB];
+        uint32_t crb = 0, nrb = 0;
+        bool cval = false, nval = false;
+        if (grp < total) fetch(grp, cu, crb, cval);
+        for (int gk = grp; gk < total; gk += kDecGroups) {
+            if (gk + kDecGroups < total) fetch(gk + kDecGroups, nu, nrb, nval);
+            const int st = gk % kSStages, kbi = gk % NKB;
             if (gk >= kSStages && !mbar_wait(&bars[kSEmpty + st], ((gk / kSStages) - 1) & 1, abort_s)) break;
-            uint8_t *a_hi = sm + L.stage + st * kStageBytes;
-            uint8_t *a_lo = a_hi + kOpTile;
-            const uint32_t rowb = (uint32_t)kr * 128;
+            tc_fence_after();
+            const uint32_t ta = tq + st * kAStageCols;
             if (kbi < DKB) {
-                // coordinates 64 kbi + 32 half + (0..31): one group of KB plane words
+                // coordinates 64 kbi + 32 h + (0..31): the KB plane words of group 2 kbi + h
+                const char *lutl = (const char *)klut + 8 * lane;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t hv[4], lo4[4];
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w[KB];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int bpos = 8 * cc + 2 * q;
-                        uint32_t idx = 0;
-#pragma unroll
-                        for (int p = 0; p < KB; ++p) idx |= ((w[p] >> bpos) & 3u) << (2 * p);
-                        const uint2 e = klut[idx];
-                        hv[q] = valid ? e.x : 0u;
-                        lo4[q] = valid ? e.y : 0u;
+                    for (int p = 0; p < KB; ++p) {
+                        const int wi = h * KB + p;
+                        w[p] = (wi & 1) ? cu[wi >> 1].y : cu[wi >> 1].x;
                     }
-                    const uint32_t off = rowb + (((uint32_t)(4 * half + cc) ^ (kr & 7)) << 4);
-                    *(uint4 *)(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                    *(uint4 *)(a_lo + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+                    uint32_t hp[16], lp[16];
+                    if (cval) {
+                        // byte k of ix[s] = table index of coordinate pair 4k + s: the pair's
+                        // two bits of plane p moved to bits 2p, 2p + 1
+                        uint32_t ix[4];
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4) {
+                            uint32_t e = 0;
+#pragma unroll
+                            for (int p = 0; p < KB; ++p) {
+                                const int sh = 2 * s4 - 2 * p;
+                                const uint32_t x = sh >= 0 ? (w[p] >> sh) : (w[p] << -sh);
+                                e |= x & (0x03030303u << (2 * p));
+                            }
+                            ix[s4] = e;
+                        }
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            // table offset idx * 256 (32 lane copies of 8 bytes per entry)
+                            const uint32_t off = __byte_perm(ix[q & 3], 0u, 0x4404u | ((uint32_t)(q >> 2) << 4));
+                            const uint2 e = *(const uint2 *)(lutl + off);
+                            hp[q] = e.x;
+                            lp[q] = e.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) hp[q] = lp[q] = 0u;
+                    }
+                    tmem_st16(ta + 32 * h, hp);
+                    tmem_st16(ta + 32 * h + 16, lp);
                 }
             } else {
-                // projections 64 (kbi - DKB) + 32 half + (0..31): one sign word, bit set = +1
+                // projections 64 (kbi - DKB) + 32 h + (0..31): +-rho 2^eA, sign bit set = +1
+                const uint32_t hv =
+                    cval ? (uint32_t)__half_as_ushort(__float2half_rn(ldexpf(f16_bits_to_f32((uint16_t)crb), eA)))
+                         : 0u;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t hv[4];
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t w = h ? cu[0].y : cu[0].x;
+                    uint32_t v[16];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t b2 = w[0] >> (8 * cc + 2 * q);
-                        // fp16 +1 is 0x3C00 and -1 is 0xBC00: the sign bit is the inverted code bit
-                        const uint32_t v = 0x3C003C00u | ((~b2 & 1u) << 15) | ((~b2 & 2u) << 30);
-                        hv[q] = valid ? v : 0u;
+                    for (int q = 0; q < 16; ++q) {
+                        const uint32_t b = ~(w >> (2 * q));
+                        v[q] = (hv | ((b & 1u) << 15)) | ((hv | ((b & 2u) << 14)) << 16);
                     }
-                    const uint32_t off = rowb + (((uint32_t)(4 * half + cc) ^ (kr & 7)) << 4);
-                    *(uint4 *)(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                    tmem_st16(ta + 32 * h, v);
                 }
             }
-            // generic-proxy stores must be visible to the tensor core (async proxy)
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kAFull + st]);
+#pragma unroll
+            for (int p = 0; p < KB; ++p) cu[p] = nu[p];
+            crb = nrb;
+            cval = nval;
         }
     } else {
         // -------------------------------------------------------- scores and top-k
+        // Each thread holds one key's scores for 32 query rows at a time (its TMEM lane) and
+        // admits those above the row's threshold into the row's queue; after the tile, thread et
+        // drains row et's queue into the row's sorted list.  A tile whose queues would overflow
+        // (the first tile, while the lists fill up, or an adversarial key order) is instead
+        // transposed through shared memory and scanned in full.
         const int q4 = warp & 3;                      // TMEM lane quarter this warp may read
         const int row = 32 * q4 + lane;               // key within the tile
-        const int et = threadIdx.x - kEpiWarp0 * 32;  // query row whose top-k this thread keeps
-        const bool et_live = rowoff[et] >= 0;
-        const float gamma = sqrtf(1.5707963267948966f) / (float)g.m;
-        const float u1 = ldexpf(1.f, -(uexp[unit * 2] + *kexp_s));
-        const float u2 = ldexpf(1.f, -uexp[unit * 2 + 1]);
-        float *mv = lv + et * (K > 0 ? K : 1);
-        int32_t *mi = li + et * (K > 0 ? K : 1);
-        float thv = -INFINITY;
-        int cnt = 0;
+        const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..127: the query row this thread drains
+        float *thr = (float *)(sm + L.thr);
+        int *qcnt = (int *)(sm + L.qcnt);
+        float *qv = (float *)(sm + L.qv);
+        int32_t *qi = (int32_t *)(sm + L.qi);
+        volatile int *ovf = (volatile int *)(sm + L.misc + 8);  // one flag per tile parity
+        const float un = ldexpf(1.f, -E);
+        float *lv = (float *)(sm + L.lv);
+        int32_t *li = (int32_t *)(sm + L.li);
+        const int ew = et >> 5;  // epilogue warp index 0..3
         for (int i = 0; i < my_tiles; ++i) {
             const int slot = i & 1;
             const int64_t t0 = (int64_t)(cidx + (int64_t)i * g.kc) * kSTile;
             const int64_t t = t0 + row;
             const bool valid = t < sp.T;
-            float c1 = 0.f, c2 = 0.f, bias = -INFINITY;
+            float c = 0.f, bias = -INFINITY;
             if (valid) {
-                const float kn = f16_bits_to_f32(sp.knorm[rec_base + t]);
-                c1 = kn * u1;
-                c2 = kn * f16_bits_to_f32(sp.krnorm[rec_base + t]) * gamma * u2;
+                c = f16_bits_to_f32(sp.knorm[rec_base + t]) * un;
                 bias = 0.f;
             }
             if (!mbar_wait(&bars[kAccFull + slot], (i >> 1) & 1, abort_s)) break;
             tc_fence_after();
-            const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16) + slot * 256;
+            const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16) + slot * kAccCols;
 #pragma unroll 1
-            for (int c = 0; c < kSTile / 32; ++c) {
-                uint32_t a1[32], a2[32];
-                tmem_ld32(tl + 32 * c, a1);
-                tmem_ld32(tl + kSTile + 32 * c, a2);
+            for (int cc = 0; cc < kSTile / 16; ++cc) {
+                uint32_t a[16];
+                tmem_ld16(tl + 16 * cc, a);
                 tmem_ld_wait();
-#pragma unroll
-                for (int l = 0; l < 32; ++l) {
-                    const float s = fmaf(c2, __uint_as_float(a2[l]), fmaf(c1, __uint_as_float(a1[l]), bias));
-                    sc[(32 * c + l) * kScStride + row] = s;
-                }
                 if (scores && valid) {
-#pragma unroll 4
-                    for (int l = 0; l < 32; ++l) {
-                        const int64_t ro = rowoff[32 * c + l];
-                        if (ro >= 0) scores[ro + t] = sc[(32 * c + l) * kScStride + row];
+#pragma unroll
+                    for (int l = 0; l < 16; ++l) {
+                        const int64_t ro = rowoff[16 * cc + l];
+                        if (ro >= 0) scores[ro + t] = fmaf(c, __uint_as_float(a[l]), bias);
                     }
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kAccEmpty + slot]);
-            if (K > 0) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (et_live) {
-                    // keys arrive in increasing index order, so a tie never displaces an entry
-                    const float *srow = sc + et * kScStride;
-#pragma unroll 8
-                    for (int kk = 0; kk < kSTile; ++kk) {
-                        const float s = srow[kk];
-                        if (s > thv) {
-                            int pos = cnt < K ? cnt : K - 1;
-                            while (pos > 0 && s > mv[pos - 1]) {
-                                mv[pos] = mv[pos - 1];
-                                mi[pos] = mi[pos - 1];
-                                --pos;
+                if (K > 0) {
+#pragma unroll
+                    for (int l4 = 0; l4 < 4; ++l4) {
+                        const float4 th = ((const float4 *)thr)[4 * cc + l4];
+                        const float tv[4] = {th.x, th.y, th.z, th.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float s = fmaf(c, __uint_as_float(a[4 * l4 + u]), bias);
+                            if (s > tv[u]) {
+                                const int r = 16 * cc + 4 * l4 + u;
+                                const int qs = atomicAdd(&qcnt[r], 1);
+                                if (qs < kQCap) {
+                                    qv[r * kQCap + qs] = s;
+                                    qi[r * kQCap + qs] = (int32_t)t;
+                                } else {
+                                    ovf[slot] = 1;
+                                }
                             }
-                            mv[pos] = s;
-                            mi[pos] = (int32_t)(t0 + kk);
-                            if (cnt < K) ++cnt;
-                            if (cnt == K) thv = mv[K - 1];
                         }
                     }
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
             }
+            if (K == 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kAccEmpty + slot]);
+                continue;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (ovf[slot] == 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kAccEmpty + slot]);
+                const int n = min(qcnt[et], kQCap);
+                if (n > 0) {
+                    float *mv = lv + et * K;
+                    int32_t *mi = li + et * K;
+#pragma unroll 1
+                    for (int j = 0; j < n; ++j) {
+                        const float sv = qv[et * kQCap + j];
+                        const int32_t ti = qi[et * kQCap + j];
+                        if (!search_better(sv, ti, mv[K - 1], mi[K - 1])) continue;
+                        int pos = K - 1;
+                        while (pos > 0 && search_better(sv, ti, mv[pos - 1], mi[pos - 1])) {
+                            mv[pos] = mv[pos - 1];
+                            mi[pos] = mi[pos - 1];
+                            --pos;
+                        }
+                        mv[pos] = sv;
+                        mi[pos] = ti;
+                    }
+                    thr[et] = mv[K - 1];
+                }
+            } else {
+                // transpose 64 query rows at a time and scan every key of the tile
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll 1
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t a[32];
+                        tmem_ld32(tl + 64 * h + 32 * cc, a);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int l = 0; l < 32; ++l)
+                            sc[(32 * cc + l) * kScStride + row] = fmaf(c, __uint_as_float(a[l]), bias);
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    // warp ew selects, for 16 of these rows, the tile's best K by K rounds of
+                    // warp arg-max, then merges them with the row's list by rank
+#pragma unroll 1
+                    for (int rr = 0; rr < 16; ++rr) {
+                        const int rl = 16 * ew + rr, r = 64 * h + rl;
+                        if (rowoff[r] < 0) continue;
+                        const float4 v4 = ((const float4 *)(sc + rl * kScStride))[lane];
+                        float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+                        float nv = -INFINITY;
+                        int32_t ni = INT32_MAX;
+                        for (int k = 0; k < K; ++k) {
+                            float bvv = -INFINITY;
+                            int32_t bii = INT32_MAX;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int32_t ix = vv[u] == -INFINITY ? INT32_MAX : (int32_t)(t0 + 4 * lane + u);
+                                if (search_better(vv[u], ix, bvv, bii)) {
+                                    bvv = vv[u];
+                                    bii = ix;
+                                }
+                            }
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) {
+                                const float ov = __shfl_xor_sync(kFull, bvv, o);
+                                const int32_t oi = __shfl_xor_sync(kFull, bii, o);
+                                if (search_better(ov, oi, bvv, bii)) {
+                                    bvv = ov;
+                                    bii = oi;
+                                }
+                            }
+                            if (lane == k) {
+                                nv = bvv;
+                                ni = bii;
+                            }
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                if (bii != INT32_MAX && (int32_t)(t0 + 4 * lane + u) == bii) vv[u] = -INFINITY;
+                        }
+                        // rank of each entry among both sorted lists (a permutation apart from
+                        // the interchangeable padding), then scatter the first K
+                        const float ev = lane < K ? lv[r * K + lane] : -INFINITY;
+                        const int32_t ei = lane < K ? li[r * K + lane] : INT32_MAX;
+                        int rn = lane, re = lane;
+                        for (int k = 0; k < K; ++k) {
+                            const float xe = __shfl_sync(kFull, ev, k), xn = __shfl_sync(kFull, nv, k);
+                            const int32_t ie = __shfl_sync(kFull, ei, k), in = __shfl_sync(kFull, ni, k);
+                            rn += search_better(xe, ie, nv, ni) ? 1 : 0;
+                            re += search_better(xn, in, ev, ei) ? 1 : 0;
+                        }
+                        __syncwarp();
+                        if (lane < K && rn < K) {
+                            lv[r * K + rn] = nv;
+                            li[r * K + rn] = ni;
+                        }
+                        if (lane < K && re < K) {
+                            lv[r * K + re] = ev;
+                            li[r * K + re] = ei;
+                        }
+                        __syncwarp();
+                        if (lane == 0) thr[r] = lv[r * K + K - 1];
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kAccEmpty + slot]);
+            }
+            qcnt[et] = 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // every thread read this parity's flag before the barrier; it is next set two tiles on
+            if (et == 0) ovf[slot] = 0;
         }
         if (K > 0) {
             const size_t base = ((size_t)blockIdx.x * kSTile + et) * K;
             for (int j = 0; j < K; ++j) {
-                cand_v[base + j] = mv[j];
-                cand_i[base + j] = mi[j];
+                cand_v[base + j] = lv[et * K + j];
+                cand_i[base + j] = li[et * K + j];
             }
         }
     }
@@ -464,10 +654,6 @@ __global__ void __launch_bounds__(kSThreads, 1)
     if (threadIdx.x == 0 && *abort_s && dev_status) atomicExch(dev_status, (int)TQ_ERR_TIMEOUT);
 }
 
-__device__ __forceinline__ bool search_better(float va, int32_t ia, float vb, int32_t ib) {
-    return va > vb || (va == vb && ia < ib);
-}
-
 // Per query row (one warp): the best K of the kc per-CTA lists, score descending, ties to the
 // smaller key index.
 __global__ void search_merge_kernel(ScoreProblem sp, SearchGeom g, int K, const float *__restrict__ cand_v,
@@ -479,10 +665,10 @@ __global__ void search_merge_kernel(ScoreProblem sp, SearchGeom g, int K, const 
     float bv[kMaxFusedTopk];
     int32_t bi[kMaxFusedTopk];
     int cnt = 0;
-    const int n = g.kc * K;
-    for (int e = threadIdx.x; e < n; e += 32) {
-        const int c = e / K, j = e % K;
-        const size_t src = (((size_t)unit * g.kc + c) * kSTile + r) * K + j;
+    const int per = K;
+    for (int e = threadIdx.x; e < g.kc * per; e += 32) {
+        const int c = e / per, j = e % per;
+        const size_t src = (((size_t)unit * g.kc + c) * kSTile + r) * per + j;
         const float v = cand_v[src];
         const int32_t ix = cand_i[src];
         if (ix == INT32_MAX) continue;
@@ -521,7 +707,7 @@ template <int KB>
 cudaError_t launch_search_kb(const Prepared &P, const ScoreProblem &sp, const SearchGeom &g, const uint8_t *qsw,
                              const int *uexp, float *scores, int K, float *cv, int32_t *ci, int32_t *dev_status,
                              cudaStream_t s) {
-    const SearchSmem L = search_smem_layout(K);
+    const SearchSmem L = search_smem_layout(K, KB);
     const size_t smem = L.total + 1024;
     auto kern = search_gemm_kernel<KB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -531,14 +717,16 @@ cudaError_t launch_search_kb(const Prepared &P, const ScoreProblem &sp, const Se
 }
 
 struct SearchScratch {
-    size_t qsw, uexp, cv, ci, total;
+    size_t qsw, umax, uexp, cv, ci, total;
 };
 
 SearchScratch search_scratch_layout(const SearchGeom &g, int topk) {
     SearchScratch S;
     size_t o = 0;
     S.qsw = o;
-    o = align_up(o + (size_t)g.units * g.nkb * 2 * kOpTile, 256);
+    o = align_up(o + (size_t)g.units * g.nkb * kStageBytes, 256);
+    S.umax = o;
+    o = align_up(o + (size_t)g.units * 2 * sizeof(unsigned), 256);
     S.uexp = o;
     o = align_up(o + (size_t)g.units * 2 * sizeof(int), 256);
     const size_t lists = (size_t)g.units * g.kc * kSTile * (topk > 0 ? topk : 0) * 4;
@@ -570,11 +758,15 @@ cudaError_t launch_search(const Prepared &P, const ScoreProblem &sp, const float
     const SearchScratch S = search_scratch_layout(g, topk);
     uint8_t *base = (uint8_t *)scratch;
     uint8_t *qsw = base + S.qsw;
+    unsigned *umax = (unsigned *)(base + S.umax);
     int *uexp = (int *)(base + S.uexp);
     float *cv = (float *)(base + S.cv);
     int32_t *ci = (int32_t *)(base + S.ci);
-    search_prep_kernel<<<g.units, 256, 0, s>>>(sp, g, qprep, qsw, uexp);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(umax, 0, (size_t)g.units * 2 * sizeof(unsigned), s);
+    if (e != cudaSuccess) return e;
+    search_max_kernel<<<dim3((unsigned)g.units, 16), 256, 0, s>>>(sp, g, qprep, umax);
+    search_tiles_kernel<<<dim3((unsigned)g.units, (unsigned)g.nkb), 256, 0, s>>>(P, sp, g, qprep, umax, qsw, uexp);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     switch (P.kbeta) {
         case 1: e = launch_search_kb<1>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;

@@ -250,6 +250,26 @@ def test_search_topk_exact_ties(tq):
         np.testing.assert_array_equal(ti[0, 0, r].cpu().numpy(), np.arange(500 * best, 500 * best + 16))
 
 
+def test_search_topk_increasing_scores(tq):
+    # scaled copies of one direction: each query's scores rise (or fall) with the key index, so
+    # every tile brings new top-k entries for half of the rows
+    import torch
+    d, m, bits, T, Nq = 128, 64, 3, 3000, 100
+    R = synth.rotation(d, 31)
+    S = synth.gaussian(m, d, 32)
+    v = synth.unit_rows(1, d, 33)
+    K = (v * (1.0 + np.arange(T, dtype=np.float32)[:, None] / T)).astype(np.float32)
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    q = synth.gaussian(Nq, d, 34).reshape(1, 1, Nq, d)
+    p = _params(tq, R, S, bits, m)
+    ora = oracle.scores(q, R, S, bits, 1, 1, 1, Nq, T, k["codes"], k["signs"], k["norm"], k["rnorm"])[0, 0]
+    for k_ in (1, 10, 16):
+        _, ti, tv = tq.tq_scores(p, torch.from_numpy(q).cuda(), _to_dev(k), 1, T, want_scores=False, topk=k_)
+        torch.cuda.synchronize()
+        for r in range(Nq):
+            check_topk(ti[0, 0, r].cpu().numpy(), tv[0, 0, r].cpu().numpy(), ora[r], k_, f"k={k_} row {r}")
+
+
 # -------------------------------------------------------------------- attend
 
 @pytest.mark.parametrize("cfg", [
