@@ -142,6 +142,8 @@ cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool 
                             int32_t *dev_status, cudaStream_t s) {
     if (compress_tc_supported(P, is_key, x_f16) && n <= (int64_t)INT32_MAX)
         return launch_compress_tc(P, is_key, x, n, codes, signs, norm, rnorm, dev_status, s);
+    if (compress_big_supported(P, is_key))
+        return launch_compress_big(P, is_key, x, x_f16, n, codes, signs, norm, rnorm, dev_status, s);
     switch (P.d) {
         case 32: return launch_npl<1>(P, is_key, x, x_f16, n, codes, signs, norm, rnorm, s);
         case 64: return launch_npl<2>(P, is_key, x, x_f16, n, codes, signs, norm, rnorm, s);

@@ -1,0 +1,577 @@
+// tq_compress_big.cu -- key / value compression on the tensor cores for any head dimension
+// d = 64 k <= 1024, fp16 or fp32 input, with both operands streamed.
+//
+// Per 128-vector tile (TurboQuantMSE.quantize / TurboQuantProd.compress; "turboquant-pytorch",
+// nav.superapi.store, 核心 API and 算法细节; atskills.one, "What It Does" stage 1 + stage 2):
+//   u = x / ||x||                          converter warps, one vector per thread: ||x|| in fp32,
+//                                          then U = u 2^10 as fp16 hi + lo, 64 coordinates per
+//                                          K-block, written into swizzled shared memory
+//   y = R u                                N-chunks of 128 outputs: ACC = U (hi + lo) x
+//                                          (R 2^8)(hi + lo), three products per k-step
+//   codes, ||y - c[idx]||                  epilogue, one vector per thread (a TMEM lane)
+//   p = S u - S' c[idx]  (S' = S R^T)      N-chunks of the projection: the S u products as above,
+//                                          then, once the tile's codes are out, K-blocks of
+//                                          -c[idx] 2^14 (hi + lo) x (S' 2^4)(hi + lo) into the
+//                                          same accumulator, so only sign(ACC) is needed
+// R is orthogonal, so ||u - R^T c|| = ||y - c||.  All products are exact in fp32 up to the
+// dropped lo x lo terms (relative 2^-22); the bucket decisions are taken on fp32 y.
+// Warp roles: 0 streams the B tiles and owns TMEM, 1 issues the MMAs, 2..5 convert the A
+// tiles, 6..9 run the epilogue.  Four TMEM slots of 128 columns keep chunks in flight.
+#include "tq_common.cuh"
+#include "tq_internal.cuh"
+#include "tq_sm100.cuh"
+
+namespace tq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBRows = 128;                   // vectors per tile (MMA M)
+constexpr int kBChunk = 128;                  // output columns per chunk (MMA N, at most)
+constexpr int kBThreads = 320;                // 10 warps
+constexpr int kCvtWarp0 = 2;                  // warps 2..5: A-tile converters
+constexpr int kBEpiWarp0 = 6;                 // warps 6..9: epilogue
+constexpr int kBStages = 3;                   // A + B operand stages
+constexpr uint32_t kATile = kBRows * 128;     // 128 x 64 fp16 (16 KB)
+constexpr uint32_t kBTileMax = kBChunk * 128; // up to 128 x 64 fp16 (16 KB)
+constexpr uint32_t kBStage = 2 * kATile + 2 * kBTileMax;  // A hi, A lo, B hi, B lo
+constexpr int kUScaleLog2 = 10;               // U = u 2^10
+constexpr int kCorrScaleLog2 = kUScaleLog2 + kRScaleLog2 - kSScaleLog2;  // correction A scale
+
+enum BBar { kBFull = 0, kBEmpty = 3, kBAccFull = 6, kBAccEmpty = 10, kBCodes = 14 };
+
+struct BigSmem {
+    uint32_t stage, ctab, bnd, cen, bars, misc, total;
+};
+
+__host__ __device__ inline BigSmem big_smem_layout() {
+    BigSmem L;
+    uint32_t o = 0;
+    L.stage = o;
+    o += kBStages * kBStage;
+    L.ctab = o;  // 16 words: fp16 hi | lo << 16 of -c[k] 2^14 (correction operand)
+    o += 16 * 4;
+    L.bnd = o;  // 16 boundaries
+    o += 16 * 4;
+    L.cen = o;  // 16 centroids
+    o += 16 * 4;
+    L.bars = o;
+    o += 32 * 8;
+    L.misc = o;
+    o += 64;
+    L.total = o;
+    return L;
+}
+
+// The chunk sequence of one tile: R chunks (rotation outputs), then, for keys, S chunks
+// (projection outputs), each with its K-blocks: d/64 over U, plus d/64 correction blocks for
+// S chunks.
+struct BigGeom {
+    int d, m, nr, ns;  // dims; number of R chunks and S chunks
+    __host__ __device__ int nchunks() const { return nr + ns; }
+    __host__ __device__ int n0(int c) const { return c < nr ? c * kBChunk : (c - nr) * kBChunk; }
+    __host__ __device__ int width(int c) const {
+        const int tot = c < nr ? d : m;
+        const int w = tot - n0(c);
+        return w < kBChunk ? w : kBChunk;
+    }
+    __host__ __device__ int nkb(int c) const { return c < nr ? d / 64 : 2 * (d / 64); }
+    __host__ __device__ int kb_per_tile() const { return nr * (d / 64) + ns * 2 * (d / 64); }
+};
+
+// Code of y against ascending boundaries b[0..2^BETA-2] (#{k : b[k] < y}) by a binary search
+// over register thresholds; t[p] receives bit p of the code.
+template <int BETA>
+__device__ __forceinline__ uint32_t big_bucket(float y, const float (&b)[16]) {
+    if constexpr (BETA == 1) {
+        return y > b[0] ? 1u : 0u;
+    } else if constexpr (BETA == 2) {
+        const uint32_t t1 = y > b[1];
+        const uint32_t t0 = y > (t1 ? b[2] : b[0]);
+        return (t1 << 1) | t0;
+    } else if constexpr (BETA == 3) {
+        const uint32_t t2 = y > b[3];
+        const uint32_t t1 = y > (t2 ? b[5] : b[1]);
+        const uint32_t t0 = y > (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]));
+        return (t2 << 2) | (t1 << 1) | t0;
+    } else {
+        const uint32_t t3 = y > b[7];
+        const uint32_t t2 = y > (t3 ? b[11] : b[3]);
+        const uint32_t t1 = y > (t3 ? (t2 ? b[13] : b[9]) : (t2 ? b[5] : b[1]));
+        const uint32_t t0 = y > (t3 ? (t2 ? (t1 ? b[14] : b[12]) : (t1 ? b[10] : b[8]))
+                                    : (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0])));
+        return (t3 << 3) | (t2 << 2) | (t1 << 1) | t0;
+    }
+}
+
+__device__ __forceinline__ uint32_t hsplit2(float a, float b, bool lo) {
+    const __half ha = __float2half_rn(a), hb = __float2half_rn(b);
+    if (!lo) return (uint32_t)__half_as_ushort(ha) | ((uint32_t)__half_as_ushort(hb) << 16);
+    const __half la = __float2half_rn(a - __half2float(ha)), lb = __float2half_rn(b - __half2float(hb));
+    return (uint32_t)__half_as_ushort(la) | ((uint32_t)__half_as_ushort(lb) << 16);
+}
+
+constexpr float kSignRecheck = 2e-4f;  // |p| below which a sign is recomputed exactly
+constexpr float kPUnscaleInv = (float)(1 << (kUScaleLog2 + kRScaleLog2));  // ACC = p 2^18
+
+// p_a = S_a . u - S'_a . c[idx] of vector v in double, one warp: lane l takes coordinates
+// l, l + 32, ...; the codes are the ones this CTA has just written for v.
+template <int BETA, bool F16>
+__device__ __noinline__ double exact_projection(const Prepared &P, const BigGeom &G, const void *xin,
+                                                const uint32_t *codes, int64_t v, int a, int lane,
+                                                const float *cen) {
+    const int d = G.d, m = G.m, KWPT = BETA * (d / 32);
+    double ss = 0.0, su = 0.0, sc = 0.0;
+    for (int j = lane; j < d; j += 32) {
+        const double xj = F16 ? (double)__half2float(((const __half *)xin)[v * d + j]) : (double)((const float *)xin)[v * d + j];
+        uint32_t idx = 0;
+#pragma unroll
+        for (int p = 0; p < BETA; ++p) idx |= ((codes[v * KWPT + (j >> 5) * BETA + p] >> lane) & 1u) << p;
+        const float c = cen[idx];
+        ss = fma(xj, xj, ss);
+        su = fma((double)P.ST[(int64_t)j * m + a], xj, su);
+        sc = fma((double)P.SpT[(int64_t)j * m + a], (double)c, sc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(kFull, ss, o);
+        su += __shfl_xor_sync(kFull, su, o);
+        sc += __shfl_xor_sync(kFull, sc, o);
+    }
+    const double nx = sqrt(ss);
+    return (nx > 0.0 ? su / nx : 0.0) - sc;
+}
+
+template <bool IS_KEY, int BETA, bool F16>
+__global__ void __launch_bounds__(kBThreads, 1)
+    compress_big_kernel(Prepared P, BigGeom G, const void *__restrict__ xin, int64_t n, uint32_t *__restrict__ codes,
+                        uint32_t *__restrict__ signs, uint16_t *__restrict__ norm, uint16_t *__restrict__ rnorm,
+                        int32_t *__restrict__ dev_status) {
+    const BigSmem L = big_smem_layout();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *bars = (uint64_t *)(sm + L.bars);
+    uint32_t *ctab = (uint32_t *)(sm + L.ctab);
+    float *bnd_s = (float *)(sm + L.bnd);
+    float *cen_s = (float *)(sm + L.cen);
+    uint32_t *tmem_s = (uint32_t *)(sm + L.misc);
+    volatile int *abort_s = (volatile int *)(sm + L.misc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d = G.d, dkb = G.d / 64;
+    const int KWPT = BETA * (d / 32);
+    const int SWPT = G.m / 32;
+    const int NC = G.nchunks();
+    const int64_t ntiles = (n + kBRows - 1) / kBRows;
+    const int my_tiles = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBStages; ++s) {
+            mbar_init(&bars[kBFull + s], 5);  // four converter warps + the B copy
+            mbar_init(&bars[kBEmpty + s], 1);
+        }
+        for (int s = 0; s < 4; ++s) {
+            mbar_init(&bars[kBAccFull + s], 1);
+            mbar_init(&bars[kBAccEmpty + s], 4);
+        }
+        for (int s = 0; s < 2; ++s) mbar_init(&bars[kBCodes + s], 4);
+        *abort_s = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 16) {
+        const int k = threadIdx.x;
+        const int K = 1 << BETA;
+        bnd_s[k] = k < K - 1 ? (IS_KEY ? P.cb->kb[k] : P.cb->vb[k]) : INFINITY;
+        const float c = k < K ? (IS_KEY ? P.cb->kc[k] : P.cb->vc[k]) : 0.f;
+        cen_s[k] = c;
+        const float cs = -c * (float)(1 << kCorrScaleLog2);
+        const __half h = __float2half_rn(cs);
+        const __half lo = __float2half_rn(cs - __half2float(h));
+        ctab[k] = (uint32_t)__half_as_ushort(h) | ((uint32_t)__half_as_ushort(lo) << 16);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_s, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_s;
+
+    if (warp == 0) {
+        // -------------------------------------------------------- B tiles (bulk copies)
+        if (lane == 0) {
+            const int wrows = IS_KEY ? d + G.m : d;
+            const uint8_t *W = (const uint8_t *)(IS_KEY ? P.RSsw : P.Rsw);
+            const size_t wlo = (size_t)wrows * d * 2;
+            const uint8_t *Sp = (const uint8_t *)P.Ssw;
+            const size_t slo = (size_t)G.m * d * 2;
+            int gk = 0, issued = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < my_tiles; ++i)
+                for (int c = 0; ok && c < NC; ++c) {
+                    const int w = G.width(c), n0 = G.n0(c), nkb = G.nkb(c);
+                    const uint32_t bytes = (uint32_t)w * 128;
+                    for (int kb = 0; kb < nkb; ++kb, ++gk) {
+                        const int st = gk % kBStages;
+                        if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint8_t *src;
+                        size_t lo;
+                        if (kb < dkb) {
+                            const int row0 = c < G.nr ? n0 : d + n0;
+                            src = W + ((size_t)kb * wrows + row0) * 128;
+                            lo = wlo;
+                        } else {
+                            src = Sp + ((size_t)(kb - dkb) * G.m + n0) * 128;
+                            lo = slo;
+                        }
+                        uint8_t *dst = sm + L.stage + st * kBStage + 2 * kATile;
+                        mbar_arrive_expect_tx(&bars[kBFull + st], 2 * bytes);
+                        bulk_load(dst, src, bytes, &bars[kBFull + st]);
+                        bulk_load(dst + kBTileMax, src + lo, bytes, &bars[kBFull + st]);
+                        issued = gk + 1;
+                    }
+                }
+            // every copy must land before the CTA can exit (bounded waits)
+            int dummy = 0;
+            for (int g = issued > kBStages ? issued - kBStages : 0; g < issued; ++g)
+                mbar_wait(&bars[kBFull + g % kBStages], (g / kBStages) & 1, (volatile int *)&dummy);
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            const uint32_t sbase = smem_u32(sm + L.stage);
+            int gk = 0, gc = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < my_tiles; ++i)
+                for (int c = 0; ok && c < NC; ++c, ++gc) {
+                    const int slot = gc & 3;
+                    if (gc >= 4 && !mbar_wait(&bars[kBAccEmpty + slot], ((gc >> 2) - 1) & 1, abort_s)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t acc = tmem + slot * kBChunk;
+                    const uint32_t idesc = idesc_f16_f32(kBRows, G.width(c));
+                    const int nkb = G.nkb(c);
+                    for (int kb = 0; kb < nkb; ++kb, ++gk) {
+                        const int st = gk % kBStages;
+                        if (!mbar_wait(&bars[kBFull + st], (gk / kBStages) & 1, abort_s)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a_hi = sbase + st * kBStage, a_lo = a_hi + kATile;
+                        const uint32_t b_hi = a_hi + 2 * kATile, b_lo = b_hi + kBTileMax;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t o = 32 * k;
+                            mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kb | k) ? 1u : 0u);
+                            mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
+                            mma_ss(acc, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
+                        }
+                        mma_commit(&bars[kBEmpty + st]);
+                    }
+                    if (ok) mma_commit(&bars[kBAccFull + slot]);
+                }
+        }
+    } else if (warp < kBEpiWarp0) {
+        // -------------------------------------------------------- A tiles, one vector per thread
+        const int r = threadIdx.x - kCvtWarp0 * 32;  // 0..127
+        const uint32_t rowb = (uint32_t)r * 128;
+        int gk = 0;
+        bool ok = true;
+        for (int i = 0; ok && i < my_tiles; ++i) {
+            const int64_t v = (blockIdx.x + (int64_t)i * gridDim.x) * kBRows + r;
+            const bool valid = v < n;
+            // ||x|| in fp32 from the input row
+            float ss = 0.f;
+            if (valid) {
+                if (F16) {
+                    const uint4 *xr = (const uint4 *)((const __half *)xin + v * d);
+                    for (int j = 0; j < d / 8; ++j) {
+                        const uint4 q = __ldg(xr + j);
+                        const uint32_t u4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __half22float2(*(const __half2 *)&u4[e]);
+                            ss = fmaf(f.x, f.x, ss);
+                            ss = fmaf(f.y, f.y, ss);
+                        }
+                    }
+                } else {
+                    const float4 *xr = (const float4 *)((const float *)xin + v * d);
+                    for (int j = 0; j < d / 4; ++j) {
+                        const float4 f = __ldg(xr + j);
+                        ss = fmaf(f.x, f.x, ss);
+                        ss = fmaf(f.y, f.y, ss);
+                        ss = fmaf(f.z, f.z, ss);
+                        ss = fmaf(f.w, f.w, ss);
+                    }
+                }
+            }
+            const float nrm = sqrtf(ss);
+            const float us = nrm > 0.f ? (float)(1 << kUScaleLog2) / nrm : 0.f;
+            if (valid) norm[v] = f32_to_f16_bits(nrm);
+            bool have_codes = false;
+            for (int c = 0; ok && c < NC; ++c) {
+                const int nkb = G.nkb(c);
+                for (int kb = 0; kb < nkb; ++kb, ++gk) {
+                    const int st = gk % kBStages;
+                    if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *ah = sm + L.stage + st * kBStage;
+                    uint8_t *al = ah + kATile;
+                    if (kb < dkb) {
+                        // U = u 2^10 for coordinates 64 kb .. 64 kb + 63, fp16 hi | lo
+#pragma unroll
+                        for (int cc = 0; cc < 8; ++cc) {
+                            float f[8];
+                            if (!valid) {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) f[e] = 0.f;
+                            } else if (F16) {
+                                const uint4 q = __ldg((const uint4 *)((const __half *)xin + v * d + 64 * kb + 8 * cc));
+                                const uint32_t u4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float2 h2 = __half22float2(*(const __half2 *)&u4[e]);
+                                    f[2 * e] = h2.x;
+                                    f[2 * e + 1] = h2.y;
+                                }
+                            } else {
+                                const float4 *xp = (const float4 *)((const float *)xin + v * d + 64 * kb + 8 * cc);
+                                const float4 p0 = __ldg(xp), p1 = __ldg(xp + 1);
+                                f[0] = p0.x; f[1] = p0.y; f[2] = p0.z; f[3] = p0.w;
+                                f[4] = p1.x; f[5] = p1.y; f[6] = p1.z; f[7] = p1.w;
+                            }
+                            uint32_t hv[4], lv4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                hv[e] = hsplit2(f[2 * e] * us, f[2 * e + 1] * us, false);
+                                lv4[e] = hsplit2(f[2 * e] * us, f[2 * e + 1] * us, true);
+                            }
+                            const uint32_t off = rowb + (((uint32_t)cc ^ (r & 7)) << 4);
+                            *(uint4 *)(ah + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                            *(uint4 *)(al + off) = make_uint4(lv4[0], lv4[1], lv4[2], lv4[3]);
+                        }
+                    } else {
+                        // correction: -c[idx] 2^14 for coordinates 64 kbc .. 64 kbc + 63 from the
+                        // tile's codes, which the epilogue has just written
+                        if (!have_codes) {
+                            if (!mbar_wait(&bars[kBCodes + (i & 1)], (i >> 1) & 1, abort_s)) {
+                                ok = false;
+                                break;
+                            }
+                            have_codes = true;
+                        }
+                        const int kbc = kb - dkb;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t w[BETA];
+#pragma unroll
+                            for (int p = 0; p < BETA; ++p)
+                                w[p] = valid ? codes[v * KWPT + (2 * kbc + h) * BETA + p] : 0u;
+#pragma unroll
+                            for (int cc = 0; cc < 4; ++cc) {
+                                uint32_t hv[4], lv4[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int l = 8 * cc + 2 * e;
+                                    uint32_t i0 = 0, i1 = 0;
+#pragma unroll
+                                    for (int p = 0; p < BETA; ++p) {
+                                        i0 |= ((w[p] >> l) & 1u) << p;
+                                        i1 |= ((w[p] >> (l + 1)) & 1u) << p;
+                                    }
+                                    const uint32_t t0 = ctab[i0], t1 = ctab[i1];
+                                    hv[e] = valid ? __byte_perm(t0, t1, 0x5410) : 0u;
+                                    lv4[e] = valid ? __byte_perm(t0, t1, 0x7632) : 0u;
+                                }
+                                const uint32_t off = rowb + (((uint32_t)(4 * h + cc) ^ (r & 7)) << 4);
+                                *(uint4 *)(ah + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                                *(uint4 *)(al + off) = make_uint4(lv4[0], lv4[1], lv4[2], lv4[3]);
+                            }
+                        }
+                    }
+                    // generic-proxy stores must be visible to the tensor core (async proxy)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[kBFull + st]);
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------- epilogue, one vector per thread
+        const int q4 = warp & 3;  // TMEM lane quarter this warp may read
+        const int r = 32 * q4 + lane;
+        float bnd_r[16], cen_r[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            bnd_r[k] = bnd_s[k];
+            cen_r[k] = cen_s[k];
+        }
+        constexpr float kYUnscale = 1.0f / (float)(1 << (kUScaleLog2 + kRScaleLog2));
+        int gc = 0;
+        bool ok = true;
+        for (int i = 0; ok && i < my_tiles; ++i) {
+            const int64_t v = (blockIdx.x + (int64_t)i * gridDim.x) * kBRows + r;
+            const bool valid = v < n;
+            float ee = 0.f;
+            for (int c = 0; c < NC; ++c, ++gc) {
+                const int slot = gc & 3;
+                if (!mbar_wait(&bars[kBAccFull + slot], (gc >> 2) & 1, abort_s)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16) + slot * kBChunk;
+                const int ng = G.width(c) / 32, g0 = G.n0(c) / 32;
+                if (c < G.nr) {
+                    // codes of rotated coordinates 32 (g0 + g) .. + 31, planar words
+#pragma unroll 1
+                    for (int g = 0; g < ng; ++g) {
+                        uint32_t a[32];
+                        tmem_ld32(tl + 32 * g, a);
+                        tmem_ld_wait();
+                        uint32_t wp[BETA];
+#pragma unroll
+                        for (int p = 0; p < BETA; ++p) wp[p] = 0u;
+#pragma unroll
+                        for (int l = 0; l < 32; ++l) {
+                            const float y = __uint_as_float(a[l]) * kYUnscale;
+                            const uint32_t idx = big_bucket<BETA>(y, bnd_r);
+#pragma unroll
+                            for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
+                            if (IS_KEY) {
+                                float cv = cen_r[0];
+#pragma unroll
+                                for (int k = 1; k < (1 << BETA); ++k) cv = idx == (uint32_t)k ? cen_r[k] : cv;
+                                const float e = y - cv;
+                                ee = fmaf(e, e, ee);
+                            }
+                        }
+                        if (valid) {
+#pragma unroll
+                            for (int p = 0; p < BETA; ++p) codes[v * KWPT + (g0 + g) * BETA + p] = wp[p];
+                        }
+                    }
+                    if (IS_KEY && c == G.nr - 1) {
+                        // every code word of this tile is out: release the correction operands
+                        if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[kBCodes + (i & 1)]);
+                    }
+                } else {
+                    // signs of the projections 32 (g0 + g) .. + 31: sign(S u - S' c) = sign(ACC).
+                    // The two terms are O(1) and cancel to p; the accumulator's rounding grows with
+                    // d (a few 1e-5 of p at d = 1024), so projections with |p| < kSignRecheck are
+                    // recomputed in double by the warp, from x, the codes, S and S'.
+                    const int64_t vbase = v - lane;
+#pragma unroll 1
+                    for (int g = 0; g < ng; ++g) {
+                        uint32_t a[32];
+                        tmem_ld32(tl + 32 * g, a);
+                        tmem_ld_wait();
+                        uint32_t sw = 0, unc = 0;
+#pragma unroll
+                        for (int l = 0; l < 32; ++l) {
+                            const float pv = __uint_as_float(a[l]);
+                            sw |= (uint32_t)(pv >= 0.f) << l;
+                            unc |= (uint32_t)(fabsf(pv) < kSignRecheck * kPUnscaleInv) << l;
+                        }
+                        if (!valid) unc = 0;
+                        uint32_t pend = __ballot_sync(kFull, unc != 0);
+                        while (pend) {
+                            const int src = __ffs(pend) - 1;
+                            pend &= pend - 1;
+                            uint32_t um = __shfl_sync(kFull, unc, src);
+                            while (um) {
+                                const int l = __ffs(um) - 1;
+                                um &= um - 1;
+                                const double pe = exact_projection<BETA, F16>(P, G, xin, codes, vbase + src,
+                                                                              32 * (g0 + g) + l, lane, cen_s);
+                                if (lane == src) sw = (sw & ~(1u << l)) | ((uint32_t)(pe >= 0.0) << l);
+                            }
+                        }
+                        if (valid) signs[v * SWPT + g0 + g] = sw;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kBAccEmpty + slot]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && *abort_s && dev_status) atomicExch(dev_status, (int)TQ_ERR_TIMEOUT);
+}
+
+template <bool IS_KEY, int BETA, bool F16>
+cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64_t n, uint32_t *codes, uint32_t *signs,
+                       uint16_t *norm, uint16_t *rnorm, int32_t *dev_status, cudaStream_t s) {
+    const BigSmem L = big_smem_layout();
+    const size_t smem = L.total + 1024;
+    auto kern = compress_big_kernel<IS_KEY, BETA, F16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t ntiles = (n + kBRows - 1) / kBRows;
+    const int grid = (int)(ntiles < sms ? ntiles : sms);
+    kern<<<grid, kBThreads, smem, s>>>(P, G, x, n, codes, signs, norm, rnorm, dev_status);
+    return cudaGetLastError();
+}
+
+template <bool IS_KEY, bool F16>
+cudaError_t launch_big_beta(const Prepared &P, const BigGeom &G, int beta, const void *x, int64_t n, uint32_t *codes,
+                            uint32_t *signs, uint16_t *norm, uint16_t *rnorm, int32_t *dev_status, cudaStream_t s) {
+    switch (beta) {
+        case 1: return launch_big<IS_KEY, 1, F16>(P, G, x, n, codes, signs, norm, rnorm, dev_status, s);
+        case 2: return launch_big<IS_KEY, 2, F16>(P, G, x, n, codes, signs, norm, rnorm, dev_status, s);
+        case 3: return launch_big<IS_KEY, 3, F16>(P, G, x, n, codes, signs, norm, rnorm, dev_status, s);
+        case 4:
+            if constexpr (!IS_KEY) return launch_big<IS_KEY, 4, F16>(P, G, x, n, codes, signs, norm, rnorm, dev_status, s);
+            return cudaErrorInvalidValue;
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool compress_big_supported(const Prepared &P, bool is_key) {
+    if (P.d < 64 || P.d > 1024 || P.d % 64) return false;
+    if (is_key && (P.m < 32 || P.m % 32)) return false;
+    return true;
+}
+
+cudaError_t launch_compress_big(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
+                                uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
+                                int32_t *dev_status, cudaStream_t s) {
+    BigGeom G;
+    G.d = P.d;
+    G.m = is_key ? P.m : 0;
+    G.nr = (P.d + kBChunk - 1) / kBChunk;
+    G.ns = is_key ? (P.m + kBChunk - 1) / kBChunk : 0;
+    const int beta = is_key ? P.kbeta : P.vbeta;
+    if (is_key)
+        return x_f16 ? launch_big_beta<true, true>(P, G, beta, x, n, codes, signs, norm, rnorm, dev_status, s)
+                     : launch_big_beta<true, false>(P, G, beta, x, n, codes, signs, norm, rnorm, dev_status, s);
+    return x_f16 ? launch_big_beta<false, true>(P, G, beta, x, n, codes, signs, norm, rnorm, dev_status, s)
+                 : launch_big_beta<false, false>(P, G, beta, x, n, codes, signs, norm, rnorm, dev_status, s);
+}
+
+}  // namespace tq

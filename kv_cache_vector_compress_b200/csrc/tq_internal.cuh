@@ -121,6 +121,10 @@ bool compress_tc_supported(const Prepared &P, bool is_key, bool x_f16);
 cudaError_t launch_compress_tc(const Prepared &P, bool is_key, const void *x, int64_t n, uint32_t *codes,
                                uint32_t *signs, uint16_t *norm, uint16_t *rnorm, int32_t *dev_status,
                                cudaStream_t s);
+bool compress_big_supported(const Prepared &P, bool is_key);
+cudaError_t launch_compress_big(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
+                                uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
+                                int32_t *dev_status, cudaStream_t s);
 cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
                             uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
                             int32_t *dev_status, cudaStream_t s);

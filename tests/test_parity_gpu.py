@@ -63,7 +63,7 @@ def test_compress_workload1(tq):
     assert len(rk) <= 2 and len(rv) <= 2
 
 
-@pytest.mark.parametrize("d", [32, 64, 128, 256])
+@pytest.mark.parametrize("d", [32, 64, 128, 256, 512, 1024])
 @pytest.mark.parametrize("n", [1, 31, 33, 257])
 @pytest.mark.parametrize("f16", [True, False])
 def test_compress_shapes(tq, d, n, f16):
@@ -77,10 +77,10 @@ def test_compress_shapes(tq, d, n, f16):
         _compress_both(tq, x, R, None, bits, False)
 
 
-def test_compress_zero_and_outlier_rows(tq):
-    d = 128
+@pytest.mark.parametrize("d", [128, 256])
+def test_compress_zero_and_outlier_rows(tq, d):
     R = synth.rotation(d, 11)
-    S = synth.gaussian(64, d, 12)
+    S = synth.gaussian(d // 2, d, 12)
     x = synth.channel_scaled_f16(96, d, 13, 14, 3)
     x[5] = 0
     x[40, :3] = np.float16(60000.0)  # near the top of the fp16 range
