@@ -15,8 +15,9 @@
 //                                          same accumulator, so only sign(ACC) is needed
 // R is orthogonal, so ||u - R^T c|| = ||y - c||.  All products are exact in fp32 up to the
 // dropped lo x lo terms (relative 2^-22); the bucket decisions are taken on fp32 y.
-// Warp roles: 0 streams the B tiles and owns TMEM, 1 issues the MMAs, 2..5 convert the A
-// tiles, 6..9 run the epilogue.  Four TMEM slots of 128 columns keep chunks in flight.
+// Warp roles: 0 streams the B tiles and owns TMEM, 1 issues the MMAs, 2..9 convert the A
+// tiles (two groups taking alternate K-blocks), 10..13 run the epilogue.  Two TMEM slots of
+// 256 columns keep one chunk's epilogue under the next chunk's MMAs.
 #include "tq_common.cuh"
 #include "tq_internal.cuh"
 #include "tq_sm100.cuh"
@@ -28,18 +29,18 @@ namespace {
 using namespace sm100;
 
 constexpr int kBRows = 128;                   // vectors per tile (MMA M)
-constexpr int kBChunk = 128;                  // output columns per chunk (MMA N, at most)
-constexpr int kBThreads = 320;                // 10 warps
-constexpr int kCvtWarp0 = 2;                  // warps 2..5: A-tile converters
-constexpr int kBEpiWarp0 = 6;                 // warps 6..9: epilogue
-constexpr int kBStages = 3;                   // A + B operand stages
+constexpr int kBChunk = 256;                  // output columns per chunk (MMA N, at most)
+constexpr int kBThreads = 448;                // 14 warps
+constexpr int kCvtWarp0 = 2;                  // warps 2..9: A-tile converters, two groups of four
+constexpr int kBEpiWarp0 = 10;                // warps 10..13: epilogue
+constexpr int kBStages = 2;                   // A + B operand stages
 constexpr uint32_t kATile = kBRows * 128;     // 128 x 64 fp16 (16 KB)
-constexpr uint32_t kBTileMax = kBChunk * 128; // up to 128 x 64 fp16 (16 KB)
+constexpr uint32_t kBTileMax = kBChunk * 128; // up to 256 x 64 fp16 (32 KB)
 constexpr uint32_t kBStage = 2 * kATile + 2 * kBTileMax;  // A hi, A lo, B hi, B lo
 constexpr int kUScaleLog2 = 10;               // U = u 2^10
 constexpr int kCorrScaleLog2 = kUScaleLog2 + kRScaleLog2 - kSScaleLog2;  // correction A scale
 
-enum BBar { kBFull = 0, kBEmpty = 3, kBAccFull = 6, kBAccEmpty = 10, kBCodes = 14 };
+enum BBar { kBFull = 0, kBEmpty = 2, kBAccFull = 4, kBAccEmpty = 6, kBCodes = 8 };
 
 struct BigSmem {
     uint32_t stage, ctab, bnd, cen, bars, misc, total;
@@ -112,26 +113,45 @@ __device__ __forceinline__ uint32_t hsplit2(float a, float b, bool lo) {
     return (uint32_t)__half_as_ushort(la) | ((uint32_t)__half_as_ushort(lb) << 16);
 }
 
-constexpr float kSignRecheck = 2e-4f;  // |p| below which a sign is recomputed exactly
+constexpr float kSignRecheck = 1e-4f;  // |p| below which a sign is recomputed exactly
 constexpr float kPUnscaleInv = (float)(1 << (kUScaleLog2 + kRScaleLog2));  // ACC = p 2^18
 
 // p_a = S_a . u - S'_a . c[idx] of vector v in double, one warp: lane l takes coordinates
-// l, l + 32, ...; the codes are the ones this CTA has just written for v.
+// 4 l + 128 i .. + 3 (row-major S and S', coalesced); the codes are the ones this CTA has just
+// written for v.
 template <int BETA, bool F16>
 __device__ __noinline__ double exact_projection(const Prepared &P, const BigGeom &G, const void *xin,
                                                 const uint32_t *codes, int64_t v, int a, int lane,
                                                 const float *cen) {
-    const int d = G.d, m = G.m, KWPT = BETA * (d / 32);
+    const int d = G.d, KWPT = BETA * (d / 32);
+    const float *sr = P.S + (int64_t)a * d, *spr = P.Sp + (int64_t)a * d;
     double ss = 0.0, su = 0.0, sc = 0.0;
-    for (int j = lane; j < d; j += 32) {
-        const double xj = F16 ? (double)__half2float(((const __half *)xin)[v * d + j]) : (double)((const float *)xin)[v * d + j];
-        uint32_t idx = 0;
+#pragma unroll 4
+    for (int j = 4 * lane; j < d; j += 128) {
+        float x4[4];
+        if (F16) {
+            const uint2 h = *(const uint2 *)((const __half *)xin + v * d + j);
+            const float2 a2 = __half22float2(*(const __half2 *)&h.x), b2 = __half22float2(*(const __half2 *)&h.y);
+            x4[0] = a2.x; x4[1] = a2.y; x4[2] = b2.x; x4[3] = b2.y;
+        } else {
+            const float4 f = *(const float4 *)((const float *)xin + v * d + j);
+            x4[0] = f.x; x4[1] = f.y; x4[2] = f.z; x4[3] = f.w;
+        }
+        const float4 s4 = *(const float4 *)(sr + j), p4 = *(const float4 *)(spr + j);
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w}, pv[4] = {p4.x, p4.y, p4.z, p4.w};
+        uint32_t w[BETA];
 #pragma unroll
-        for (int p = 0; p < BETA; ++p) idx |= ((codes[v * KWPT + (j >> 5) * BETA + p] >> lane) & 1u) << p;
-        const float c = cen[idx];
-        ss = fma(xj, xj, ss);
-        su = fma((double)P.ST[(int64_t)j * m + a], xj, su);
-        sc = fma((double)P.SpT[(int64_t)j * m + a], (double)c, sc);
+        for (int p = 0; p < BETA; ++p) w[p] = codes[v * KWPT + (j >> 5) * BETA + p] >> (j & 31);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t idx = 0;
+#pragma unroll
+            for (int p = 0; p < BETA; ++p) idx |= ((w[p] >> e) & 1u) << p;
+            const double xj = (double)x4[e];
+            ss = fma(xj, xj, ss);
+            su = fma((double)sv[e], xj, su);
+            sc = fma((double)pv[e], (double)cen[idx], sc);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -168,10 +188,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kBStages; ++s) {
-            mbar_init(&bars[kBFull + s], 5);  // four converter warps + the B copy
+            mbar_init(&bars[kBFull + s], 5);  // the four converter warps of a group + the B copy
             mbar_init(&bars[kBEmpty + s], 1);
         }
-        for (int s = 0; s < 4; ++s) {
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[kBAccFull + s], 1);
             mbar_init(&bars[kBAccEmpty + s], 4);
         }
@@ -249,8 +269,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
             bool ok = true;
             for (int i = 0; ok && i < my_tiles; ++i)
                 for (int c = 0; ok && c < NC; ++c, ++gc) {
-                    const int slot = gc & 3;
-                    if (gc >= 4 && !mbar_wait(&bars[kBAccEmpty + slot], ((gc >> 2) - 1) & 1, abort_s)) {
+                    const int slot = gc & 1;
+                    if (gc >= 2 && !mbar_wait(&bars[kBAccEmpty + slot], ((gc >> 1) - 1) & 1, abort_s)) {
                         ok = false;
                         break;
                     }
@@ -281,7 +301,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
     } else if (warp < kBEpiWarp0) {
         // -------------------------------------------------------- A tiles, one vector per thread
-        const int r = threadIdx.x - kCvtWarp0 * 32;  // 0..127
+        const int cg = (warp - kCvtWarp0) >> 2;           // group: K-block steps gk with gk % 2 == cg
+        const int r = (threadIdx.x - kCvtWarp0 * 32) & 127;  // the vector this thread converts
         const uint32_t rowb = (uint32_t)r * 128;
         int gk = 0;
         bool ok = true;
@@ -316,29 +337,35 @@ __global__ void __launch_bounds__(kBThreads, 1)
             }
             const float nrm = sqrtf(ss);
             const float us = nrm > 0.f ? (float)(1 << kUScaleLog2) / nrm : 0.f;
-            if (valid) norm[v] = f32_to_f16_bits(nrm);
+            if (valid && cg == 0) norm[v] = f32_to_f16_bits(nrm);
             bool have_codes = false;
             for (int c = 0; ok && c < NC; ++c) {
                 const int nkb = G.nkb(c);
                 for (int kb = 0; kb < nkb; ++kb, ++gk) {
+                    if ((gk & 1) != cg) continue;
                     const int st = gk % kBStages;
-                    if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
-                        ok = false;
-                        break;
-                    }
                     uint8_t *ah = sm + L.stage + st * kBStage;
                     uint8_t *al = ah + kATile;
                     if (kb < dkb) {
-                        // U = u 2^10 for coordinates 64 kb .. 64 kb + 63, fp16 hi | lo
+                        // U = u 2^10 for coordinates 64 kb .. 64 kb + 63, fp16 hi | lo; the inputs
+                        // are fetched before waiting for the stage to free up
+                        constexpr int NQ = F16 ? 8 : 16;
+                        uint4 q[NQ];
+#pragma unroll
+                        for (int e = 0; e < NQ; ++e) {
+                            q[e] = make_uint4(0u, 0u, 0u, 0u);
+                            if (valid)
+                                q[e] = __ldg((const uint4 *)((const char *)xin + (v * d + 64 * kb) * (F16 ? 2 : 4)) + e);
+                        }
+                        if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
+                            ok = false;
+                            break;
+                        }
 #pragma unroll
                         for (int cc = 0; cc < 8; ++cc) {
                             float f[8];
-                            if (!valid) {
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) f[e] = 0.f;
-                            } else if (F16) {
-                                const uint4 q = __ldg((const uint4 *)((const __half *)xin + v * d + 64 * kb + 8 * cc));
-                                const uint32_t u4[4] = {q.x, q.y, q.z, q.w};
+                            if (F16) {
+                                const uint32_t u4[4] = {q[cc].x, q[cc].y, q[cc].z, q[cc].w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     const float2 h2 = __half22float2(*(const __half2 *)&u4[e]);
@@ -346,10 +373,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
                                     f[2 * e + 1] = h2.y;
                                 }
                             } else {
-                                const float4 *xp = (const float4 *)((const float *)xin + v * d + 64 * kb + 8 * cc);
-                                const float4 p0 = __ldg(xp), p1 = __ldg(xp + 1);
-                                f[0] = p0.x; f[1] = p0.y; f[2] = p0.z; f[3] = p0.w;
-                                f[4] = p1.x; f[5] = p1.y; f[6] = p1.z; f[7] = p1.w;
+                                const uint4 a0 = q[2 * cc], a1 = q[2 * cc + 1];
+                                f[0] = __uint_as_float(a0.x); f[1] = __uint_as_float(a0.y);
+                                f[2] = __uint_as_float(a0.z); f[3] = __uint_as_float(a0.w);
+                                f[4] = __uint_as_float(a1.x); f[5] = __uint_as_float(a1.y);
+                                f[6] = __uint_as_float(a1.z); f[7] = __uint_as_float(a1.w);
                             }
                             uint32_t hv[4], lv4[4];
 #pragma unroll
@@ -372,12 +400,18 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             have_codes = true;
                         }
                         const int kbc = kb - dkb;
+                        uint32_t w[2][BETA];
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t w[BETA];
+                        for (int h = 0; h < 2; ++h)
 #pragma unroll
                             for (int p = 0; p < BETA; ++p)
-                                w[p] = valid ? codes[v * KWPT + (2 * kbc + h) * BETA + p] : 0u;
+                                w[h][p] = valid ? codes[v * KWPT + (2 * kbc + h) * BETA + p] : 0u;
+                        if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
+                            ok = false;
+                            break;
+                        }
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
 #pragma unroll
                             for (int cc = 0; cc < 4; ++cc) {
                                 uint32_t hv[4], lv4[4];
@@ -387,8 +421,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
                                     uint32_t i0 = 0, i1 = 0;
 #pragma unroll
                                     for (int p = 0; p < BETA; ++p) {
-                                        i0 |= ((w[p] >> l) & 1u) << p;
-                                        i1 |= ((w[p] >> (l + 1)) & 1u) << p;
+                                        i0 |= ((w[h][p] >> l) & 1u) << p;
+                                        i1 |= ((w[h][p] >> (l + 1)) & 1u) << p;
                                     }
                                     const uint32_t t0 = ctab[i0], t1 = ctab[i1];
                                     hv[e] = valid ? __byte_perm(t0, t1, 0x5410) : 0u;
@@ -425,8 +459,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
             const bool valid = v < n;
             float ee = 0.f;
             for (int c = 0; c < NC; ++c, ++gc) {
-                const int slot = gc & 3;
-                if (!mbar_wait(&bars[kBAccFull + slot], (gc >> 2) & 1, abort_s)) {
+                const int slot = gc & 1;
+                if (!mbar_wait(&bars[kBAccFull + slot], (gc >> 1) & 1, abort_s)) {
                     ok = false;
                     break;
                 }

@@ -35,6 +35,8 @@ struct WsLayout {
     size_t Rsw;        // fp16 hi | lo of R * 2^kRScaleLog2, tensor-core operand layout
     size_t Ssw;        // fp16 hi | lo of (S R^T) * 2^kSScaleLog2, same layout
     size_t RSsw;       // fp16 hi | lo of [R; S] * 2^kRScaleLog2 (d + m rows), same layout
+    size_t S;          // fp32 [m, d]      copy of S
+    size_t Sp;         // fp32 [m, d]      S R^T
     size_t total;
 };
 
@@ -81,6 +83,10 @@ inline WsLayout ws_layout(int d, int m) {
     o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * (m > 0 ? m : 1), 1024);
     L.RSsw = o;
     o = align_up(o + 2 * sizeof(uint16_t) * (size_t)d * (d + m), 1024);
+    L.S = o;
+    o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 256);
+    L.Sp = o;
+    o = align_up(o + sizeof(float) * (size_t)d * (m > 0 ? m : 1), 256);
     L.total = o;
     return L;
 }
@@ -89,7 +95,7 @@ inline WsLayout ws_layout(int d, int m) {
 struct Prepared {
     int d, m, kbeta, vbeta;
     const Codebooks *cb;
-    const float *R, *RT, *ST, *SpT;
+    const float *R, *RT, *ST, *SpT, *S, *Sp;
     const uint16_t *Rsw, *Ssw, *RSsw;
 };
 
@@ -109,6 +115,8 @@ inline Prepared prepared_view(const tq_params *p) {
     v.Rsw = (const uint16_t *)(w + L.Rsw);
     v.Ssw = (const uint16_t *)(w + L.Ssw);
     v.RSsw = (const uint16_t *)(w + L.RSsw);
+    v.S = (const float *)(w + L.S);
+    v.Sp = (const float *)(w + L.Sp);
     return v;
 }
 

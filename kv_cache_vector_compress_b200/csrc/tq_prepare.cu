@@ -49,9 +49,12 @@ __global__ void prepare_kernel(const float *__restrict__ R, const float *__restr
         }
     }
     if (m <= 0) return;
+    float *Srow = (float *)(ws + L.S);
+    float *Sprow = (float *)(ws + L.Sp);
     for (int64_t e = tid; e < (int64_t)m * d; e += nth) {
         int a = (int)(e / d), j = (int)(e % d);
         ST[(int64_t)j * m + a] = S[e];
+        Srow[e] = S[e];
     }
     // S' = S R^T expressed on rotated coordinates: S'[a][i] = sum_k S[a][k] R[i][k],
     // accumulated in double and rounded once.
@@ -62,6 +65,7 @@ __global__ void prepare_kernel(const float *__restrict__ R, const float *__restr
         double acc = 0.0;
         for (int k = 0; k < d; ++k) acc += (double)sr[k] * (double)rr[k];
         SpT[(int64_t)i * m + a] = (float)acc;
+        Sprow[e] = (float)acc;
         // split operand of S' * 2^s: row a = projection index, k = i (rotated coordinate)
         const double sv = acc * (double)(1 << kSScaleLog2);
         const __half hi = __double2half(sv);
