@@ -421,6 +421,7 @@ def run_workload(args):
         name = "Qwen2.5-3B-shaped prefill compress: 36 layers x 2 KV heads x 8192 x 128 fp16, bits 2/3/4"
     elif wl == 4:
         d, m, B, Hq, Hkv, T = 256, 128, 8, 16, 4, 65536
+        B = args.batch if args.batch > 0 else B
         n = B * Hkv * T
         R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
         S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
@@ -444,7 +445,8 @@ def run_workload(args):
             out.append(rec(f"attend_b{bits}", ms, n, "keys", n * (kb + vb)))
         name = "wide-head decode: B8 Hq16/Hkv4 T65536 d256 m128, bits 2 and 4, 1% key channels x20"
     elif wl == 5:
-        d, m, bits, N, Nq, k = 1024, 512, 4, 1_000_000, 1024, 10
+        d, m, bits, Nq, k = 1024, 512, 4, 1024, 10
+        N = args.db if args.db > 0 else 1_000_000
         R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
         S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
         p = tq.Params(d, bits, m, R, S)
@@ -469,7 +471,7 @@ def run_workload(args):
         r["tflops_mma"] = 2.0 * pad(Nq) * pad(N) * (3 * d + 2 * m) / (ms * 1e-3) / 1e12
         r["frac_tensor"] = r["tflops_mma"] / pk["bf16_tflops"] if pk.get("bf16_tflops") else None
         out.append(r)
-        name = "vector search: 1M x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
+        name = f"vector search: {N} x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
     else:
         raise SystemExit("unknown workload")
     print(json.dumps({"workload": wl, "name": name, "ops": out, "peak_hbm_gbs": pk["hbm_gbs"]}), flush=True)
@@ -484,6 +486,8 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's 32)")
+    ap.add_argument("--db", type=int, default=0,
+                    help="database vectors of the vector-search workload (default 1,000,000; smaller for profiling)")
     ap.add_argument("--workload", type=int, default=3,
                     help="3 (default) prints the headline line; 1, 2, 4, 5 print secondary per-op measurements")
     args = ap.parse_args()
