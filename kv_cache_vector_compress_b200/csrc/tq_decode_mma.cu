@@ -114,12 +114,15 @@ struct MmaSmem {
 __host__ __device__ inline MmaSmem mma_smem_layout(int D, int KB, int VB, int m) {
     MmaSmem L;
     uint32_t o = 0;
+    // 64-entry pair tables get one copy per lane (entry e of lane l at e * 256 + 8 l), so a
+    // warp's random look-ups never conflict; smaller tables fit one bank row and the 256-entry
+    // one stays shared
     L.klut = o;
-    o += 64 * 8;
+    o += KB == 3 ? 64 * 32 * 8 : 64 * 8;
     L.slut = o;
     o += 16 * 4;
     L.vlut = o;
-    o += 256 * 8;
+    o += VB == 3 ? 64 * 32 * 8 : 256 * 8;
     L.rowsc = o;
     o += 2 * kRowsPerCta * 4;
     L.ptile = o;
@@ -187,22 +190,25 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
         for (int k = 0; k < (1 << VB); ++k) vmax = fmaxf(vmax, fabsf(P.cb->vc[k]));
     const int ek = scale_exp(kmax), ev = scale_exp(vmax);
     const float ksc = ldexpf(1.f, ek), vsc = ldexpf(1.f, ev);
-    for (int e = tid; e < (1 << (2 * KB)); e += kThreadsMma) {
+    constexpr int KCOPIES = KB == 3 ? 32 : 1, VCOPIES = VB == 3 ? 32 : 1;
+    for (int ec = tid; ec < (1 << (2 * KB)) * KCOPIES; ec += kThreadsMma) {
         // index bits: plane p of (coordinate j, coordinate j+1) at bits (2p, 2p+1)
+        const int e = ec / KCOPIES;
         int i0 = 0, i1 = 0;
         for (int p = 0; p < KB; ++p) {
             i0 |= ((e >> (2 * p)) & 1) << p;
             i1 |= ((e >> (2 * p + 1)) & 1) << p;
         }
         const float a0 = P.cb->kc[i0] * ksc, a1 = P.cb->kc[i1] * ksc;
-        klut[e] = make_uint2(pack_h2(a0, a1), pack_h2(a0 - hi_part(a0), a1 - hi_part(a1)));
+        klut[ec] = make_uint2(pack_h2(a0, a1), pack_h2(a0 - hi_part(a0), a1 - hi_part(a1)));
     }
     if (tid < 4) slut[tid] = pack_h2((tid & 1) ? 1.f : -1.f, (tid & 2) ? 1.f : -1.f);
     if (ATTEND) {
-        for (int e = tid; e < (1 << (2 * VB)); e += kThreadsMma) {
+        for (int ec = tid; ec < (1 << (2 * VB)) * VCOPIES; ec += kThreadsMma) {
             // low VB bits: token 2i, next VB bits: token 2i+1 (same coordinate); hi and lo fp16 parts
+            const int e = ec / VCOPIES;
             const float a0 = P.cb->vc[e & ((1 << VB) - 1)] * vsc, a1 = P.cb->vc[e >> VB] * vsc;
-            vlut[e] = make_uint2(pack_h2(a0, a1), pack_h2(a0 - hi_part(a0), a1 - hi_part(a1)));
+            vlut[ec] = make_uint2(pack_h2(a0, a1), pack_h2(a0 - hi_part(a0), a1 - hi_part(a1)));
         }
     }
     if (tid < kRowsPerCta) {
@@ -335,7 +341,8 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
                         uint32_t ah[4], al[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const uint2 e = lut64(klut, KSH == 3 ? o[u] : (o[u] << 1));
+                            const uint2 e = KCOPIES > 1 ? lut64(klut, (o[u] << 6) + 8 * lane)
+                                                        : lut64(klut, KSH == 3 ? o[u] : (o[u] << 1));
                             ah[u] = e.x;
                             al[u] = e.y;
                         }
@@ -484,7 +491,8 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
                         uint32_t al[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const uint2 e = lut64(vlut, VSH ? (o4[u] << 1) : (o4[u] << 3));
+                            const uint2 e = VCOPIES > 1 ? lut64(vlut, (o4[u] << 6) + 8 * lane)
+                                                        : lut64(vlut, VSH ? (o4[u] << 1) : (o4[u] << 3));
                             a[u] = e.x;
                             al[u] = e.y;
                         }
