@@ -182,6 +182,20 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
                     int32_t *dev_status, tq_stream_t stream);
 
 /*
+ * tq_selftest_wait_timeout -- exercises the device-side failure path of every kernel.
+ * (The pages have no counterpart: this is a diagnostic of the library.)
+ * Every wait of the kernels on another warp or on a copy is bounded; when one runs out, the
+ * kernel records TQ_ERR_TIMEOUT in dev_status, drains its copies, frees its tensor memory and
+ * returns, so the context stays usable.  This call launches one small kernel whose wait can only
+ * end by its time limit (a barrier nothing ever arrives at) and so must leave TQ_ERR_TIMEOUT in
+ * *dev_status after about timeout_ms milliseconds.
+ *   dev_status : device int32 (required); set, never cleared
+ *   timeout_ms : 1 .. 10000, else TQ_ERR_INVALID_ARG
+ * Returns TQ_OK once the kernel is enqueued on stream.
+ */
+tq_status tq_selftest_wait_timeout(int32_t *dev_status, uint32_t timeout_ms, tq_stream_t stream);
+
+/*
  * tq_attend_static -- tq_attend for callers that cannot allocate device memory when they call.
  * (The pages have no counterpart: this is an addition of the library.)
  * A serving loop whose device memory is all handed to its own pool up front, or code that must

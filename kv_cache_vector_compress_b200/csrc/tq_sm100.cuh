@@ -55,19 +55,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns false) when
-// *abort is set by another thread or after kTimeoutNs, in which case it sets *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// *abort is set by another thread or after timeout_ns, in which case it sets *abort.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                             uint64_t timeout_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
+        if (globaltimer() - t0 > timeout_ns) {
             *abort = 1;
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait_ns(bar, parity, abort, kTimeoutNs);
 }
 
 // --------------------------------------------------------------- bulk copies

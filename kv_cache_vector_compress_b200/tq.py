@@ -65,12 +65,14 @@ _lib.tq_attend.restype = _I
 _lib.tq_attend_static.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P,
                                   _P, _P]
 _lib.tq_attend_static.restype = _I
+_lib.tq_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint32, _P]
+_lib.tq_selftest_wait_timeout.restype = _I
 
 TQ_STATIC_SCRATCH_BYTES = 16 << 20
 
 EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_workspace_bytes", "tq_prepare",
            "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores",
-           "tq_attend_scratch_bytes", "tq_attend", "tq_attend_static"]
+           "tq_attend_scratch_bytes", "tq_attend", "tq_selftest_wait_timeout", "tq_attend_static"]
 
 
 class TQError(RuntimeError):
@@ -245,3 +247,10 @@ def tq_attend_static(p: Params, q: torch.Tensor, keys, values, Hkv: int, T: int,
                                  _ptr(vc), _ptr(vn), float(scale), _ptr(out), _ptr(dev_status), _stream()),
            "tq_attend_static")
     return out
+
+
+def tq_selftest_wait_timeout(dev_status: torch.Tensor, timeout_ms: int = 100):
+    """Launch the library's bounded-wait self-test: a kernel whose wait can only end by its time
+    limit, which must leave TQ_ERR_TIMEOUT in dev_status (a device int32 tensor)."""
+    _check(_lib.tq_selftest_wait_timeout(_ptr(dev_status), timeout_ms, _stream()), "tq_selftest_wait_timeout")
+
