@@ -108,7 +108,8 @@ __device__ __forceinline__ void stage_copy(uint32_t *dst, const uint32_t *src, i
 
 struct MmaSmem {
     uint32_t klut, slut, vlut, rowsc, ptile, stage, total;
-    uint32_t stage_bytes, kc, ks, vc;
+    uint32_t stage_bytes, kc, ks, vc, kn, kr, vn;
+    int nst;  // stages in each warp's ring
 };
 
 __host__ __device__ inline MmaSmem mma_smem_layout(int D, int KB, int VB, int m) {
@@ -132,9 +133,16 @@ __host__ __device__ inline MmaSmem mma_smem_layout(int D, int KB, int VB, int m)
     L.kc = 0;
     L.ks = L.kc + kWarpStage * KB * g32 * 4;
     L.vc = L.ks + kWarpStage * (m / 32) * 4;
-    L.stage_bytes = (L.vc + kWarpStage * VB * g32 * 4 + 15) & ~15u;
+    // per-token fp16 norms: key, key residual, value; copied in 4-byte words from an even
+    // record index, so one extra element on each side
+    const uint32_t nb = ((kWarpStage + 2) * 2 + 15) & ~15u;
+    L.kn = (L.vc + kWarpStage * VB * g32 * 4 + 15) & ~15u;
+    L.kr = L.kn + nb;
+    L.vn = L.kr + nb;
+    L.stage_bytes = L.vn + nb;
+    L.nst = 4 * 4 * L.stage_bytes <= 64u * 1024 ? 4 : 2;
     L.stage = o;
-    o += 4 * 2 * L.stage_bytes;  // 4 warps x 2 stages
+    o += 4 * L.nst * L.stage_bytes;  // 4 warps x nst stages
     const uint32_t comb = 4u * kRowsPerCta * (D + 2) * 4;
     if (o < L.stage + comb) o = L.stage + comb;
     L.total = o;
@@ -264,49 +272,55 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     const int64_t wlen = (((t1 - t0) + 4 * 16 - 1) / (4 * 16)) * 16;
     const int64_t wt0 = min(t1, t0 + warp * wlen);
     const int64_t wt1 = min(t1, wt0 + wlen);
-    uint8_t *wstage = smem + L.stage + (size_t)warp * 2 * L.stage_bytes;
+    const int NST = L.nst;
+    uint8_t *wstage = smem + L.stage + (size_t)warp * NST * L.stage_bytes;
     const int64_t rec_base = sl * sp.T;
+    const int64_t nrec = (int64_t)sp.B * sp.Hkv * sp.T;
+    // fp16 norms of records [rec0, rec0 + ntok): 4-byte words from the even index below rec0; an
+    // odd last element that would take its word past the end of the arrays is copied directly
+    auto stage_norms = [&](uint16_t *dst, const uint16_t *src, int64_t rec0, int ntok) {
+        const int64_t e0 = rec0 & ~(int64_t)1;
+        const int64_t e1 = rec0 + ntok;
+        const int words = (int)((e1 - e0) >> 1);
+        for (int i = lane; i < words; i += 32) cp_async<4>((uint32_t *)dst + i, (const uint32_t *)(src + e0) + i);
+        if (((e1 - e0) & 1) && lane == 0) {
+            if (e1 + 1 <= nrec) cp_async<4>((uint32_t *)dst + words, (const uint32_t *)(src + e0) + words);
+            else dst[2 * words] = src[e1 - 1];
+        }
+    };
     auto issue = [&](int s) {
         const int64_t tb = wt0 + (int64_t)s * kWarpStage;
         if (tb < wt1) {
             const int ntok = (int)min((int64_t)kWarpStage, wt1 - tb);
-            uint8_t *st = wstage + (s & 1) * L.stage_bytes;
+            uint8_t *st = wstage + (s % NST) * L.stage_bytes;
             const int64_t rec0 = rec_base + tb;
             stage_copy<KWPT>((uint32_t *)(st + L.kc), sp.kcodes + rec0 * KWPT, ntok * KWPT, lane);
             stage_copy<SW>((uint32_t *)(st + L.ks), sp.ksigns + rec0 * SW, ntok * SW, lane);
             if (ATTEND) stage_copy<VWPT>((uint32_t *)(st + L.vc), sp.vcodes + rec0 * VWPT, ntok * VWPT, lane);
+            stage_norms((uint16_t *)(st + L.kn), sp.knorm, rec0, ntok);
+            stage_norms((uint16_t *)(st + L.kr), sp.krnorm, rec0, ntok);
+            if (ATTEND) stage_norms((uint16_t *)(st + L.vn), sp.vnorm, rec0, ntok);
         }
         cp_async_commit();
     };
-    // norms of the thread's two tokens (gid, gid+8) of a 16-token block
-    float nka = 0.f, nkb = 0.f, nra = 0.f, nrb = 0.f, nva = 0.f, nvb = 0.f;
-    auto load_norms = [&](int64_t gtb) {
-        const int64_t ta = gtb + gid, tb = gtb + gid + 8;
-        if (ta < wt1) {
-            nka = f16_bits_to_f32(sp.knorm[rec_base + ta]);
-            nra = f16_bits_to_f32(sp.krnorm[rec_base + ta]);
-            if (ATTEND) nva = f16_bits_to_f32(sp.vnorm[rec_base + ta]);
-        }
-        if (tb < wt1) {
-            nkb = f16_bits_to_f32(sp.knorm[rec_base + tb]);
-            nrb = f16_bits_to_f32(sp.krnorm[rec_base + tb]);
-            if (ATTEND) nvb = f16_bits_to_f32(sp.vnorm[rec_base + tb]);
-        }
-    };
-
     float oacc[ATTEND ? KSTEP : 1][4];
 #pragma unroll
     for (int c = 0; c < (ATTEND ? KSTEP : 1); ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
     float M0 = -INFINITY, M1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
     const int nstages = (int)((wt1 - wt0 + kWarpStage - 1) / kWarpStage);
-    issue(0);
-    issue(1);
-    load_norms(wt0);
+    for (int k = 0; k < NST - 1; ++k) issue(k);
     for (int s = 0; s < nstages; ++s) {
-        cp_async_wait<1>();
+        // the slot of stage s + NST - 1 was last read in iteration s - 1 (synchronised below)
+        issue(s + NST - 1);
+        if (NST == 4) cp_async_wait<3>();
+        else cp_async_wait<1>();
         __syncwarp();
-        const uint8_t *st = wstage + (s & 1) * L.stage_bytes;
+        const uint8_t *st = wstage + (s % NST) * L.stage_bytes;
+        const int noff = (int)((rec_base + wt0 + (int64_t)s * kWarpStage) & 1);
+        const uint16_t *skn = (const uint16_t *)(st + L.kn) + noff;
+        const uint16_t *skr = (const uint16_t *)(st + L.kr) + noff;
+        const uint16_t *svn = (const uint16_t *)(st + L.vn) + noff;
         const uint32_t *skc = (const uint32_t *)(st + L.kc);
         const uint32_t *sks = (const uint32_t *)(st + L.ks);
         const uint32_t *svc = (const uint32_t *)(st + L.vc);
@@ -317,8 +331,11 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
             if (gtb >= wt1) break;
             const int ta = ob + gid, tb8 = ob + gid + 8;
             const bool va = gtb + gid < wt1, vb = gtb + gid + 8 < wt1;
-            const float kna = nka, knb = nkb, rna = nra * gamma, rnb = nrb * gamma, vna = nva, vnb = nvb;
-            load_norms(gtb + 16);  // next block's norms, in flight during this block
+            const float kna = va ? f16_bits_to_f32(skn[ta]) : 0.f, knb = vb ? f16_bits_to_f32(skn[tb8]) : 0.f;
+            const float rna = va ? f16_bits_to_f32(skr[ta]) * gamma : 0.f;
+            const float rnb = vb ? f16_bits_to_f32(skr[tb8]) * gamma : 0.f;
+            const float vna = (ATTEND && va) ? f16_bits_to_f32(svn[ta]) : 0.f;
+            const float vnb = (ATTEND && vb) ? f16_bits_to_f32(svn[tb8]) : 0.f;
             // ---------------- scores
             float cs[4] = {0.f, 0.f, 0.f, 0.f}, cd[4] = {0.f, 0.f, 0.f, 0.f};
             {
@@ -523,7 +540,6 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
             }
         }
         __syncwarp();
-        issue(s + 2);
     }
     cp_async_wait<0>();
     if constexpr (!ATTEND) return;
