@@ -5,13 +5,16 @@
 //   rotation    ACC[v, j] = sum_i X[v, i] (R_hi + R_lo)[j, i]          tcgen05, smem x smem
 //               (X is the fp16 input tile, exact in fp16; R * 2^8 = R_hi + R_lo in fp16, so
 //               the product carries ~22 bits of R and the accumulator is fp32)
-//   epilogue    n = ||ACC row|| (R orthogonal), y = ACC / n, idx = code of y, planar pack,
-//               keys: e = y - c[idx] split into fp16 hi + lo, written back into TMEM
+//   code step   n = ||x|| (from the input tile), y = ACC / (2^8 n), idx = code of y, planar pack;
+//               keys: e = 2^14 (y - c[idx]) split into fp16 hi + lo, written back into TMEM
 //   projection  P[v, a] = sum_j (E_hi (S'_hi + S'_lo) + E_lo S'_hi)[v, j]   tcgen05, tmem x smem
-//               with S' = S R^T (so P = S r for the residual r = R^T e); sign bits of P.
-// One thread of the epilogue owns one vector (one TMEM lane), so norms and residual norms are
-// thread-local.  Warp roles: warp 0 loads (TMA) and owns TMEM, warp 1 issues the MMAs, two
-// groups of four epilogue warps take alternate tiles, each with its own half of TMEM.
+//               with S' = S R^T, so P is a positive multiple of S r for the residual r = R^T e;
+//   sign step   QJL sign bits of P.
+// One thread owns one vector (one TMEM lane) and half of its coordinates.  Warp roles: warp 0
+// loads (TMA) and owns TMEM, warp 1 issues the MMAs, warps 2..9 run the code and sign steps of
+// every tile, warps 10..11 take the row norms.  TMEM holds up to four rotation accumulators
+// (keys: three beside two projection accumulators), so the rotation of later tiles and the
+// projection of earlier ones keep the tensor cores busy while a tile is being coded.
 #include <cudaTypedefs.h>
 
 #include "tq_common.cuh"
@@ -28,46 +31,60 @@ constexpr int kTileRows = 128;
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kEpiWarp0 = 2;   // warps 2..9: epilogue (two groups of four)
 constexpr int kNormWarp0 = 10; // warps 10..11: row norms of the input tiles
-constexpr int kCScaleLog2 = 10;  // centroid scale before the fp16 hi/lo split
+constexpr int kEScaleLog2 = 14;  // residual scale before the fp16 hi/lo split
 
 struct TcSmem {
     // offsets from the 1024-aligned dynamic shared memory base
     uint32_t R, S, X, bars, misc;
     uint32_t total;
-    int nst;
+    int nst;  // input stages
+    int nrs;  // rotation accumulators in TMEM
 };
+
+// Rotation accumulators (D columns each) that fit in the 512 TMEM columns beside the keys' two
+// projection accumulators (m columns each); at most four.
+__host__ __device__ inline int tc_rotation_slots(int D, int m, bool is_key) {
+    const int r = is_key ? (512 - 2 * m) / D : 512 / D;
+    return r > 4 ? 4 : r;
+}
+
+// misc block: codebook and flags (256 B), squared row norms [4][128], half residual norms [4][128]
+constexpr uint32_t kMiscNorm = 256, kMiscEe = 256 + 2048;
+constexpr uint32_t kMiscBytes = kMiscEe + 2048;
 
 __host__ __device__ inline TcSmem tc_smem_layout(int D, int m, bool is_key) {
     TcSmem L;
     uint32_t o = 0;
     L.R = o;
-    o += 2u * (is_key ? D + m : D) * D * 2;  // [R; S] (keys) or R (values), hi | lo
+    o += 2u * D * D * 2;  // R hi | lo
     L.S = o;
-    if (is_key) o += 2u * m * D * 2;
+    if (is_key) o += 2u * m * D * 2;  // S' = S R^T, hi | lo
     L.X = o;
     const uint32_t xs = kTileRows * D * 2;
-    uint32_t budget = 225u * 1024 - o - 2048;
+    const uint32_t budget = 225u * 1024 - o - 256 - kMiscBytes;
     int nst = (int)(budget / xs);
     if (nst > 4) nst = 4;
     L.nst = nst;
+    L.nrs = tc_rotation_slots(D, m, is_key);
     o += nst * xs;
     L.bars = o;
     o += 256;
     L.misc = o;
-    o += 2048;
+    o += kMiscBytes;
     L.total = o;
     return L;
 }
 
 enum BarIdx {
     kOpnd = 0,
-    kFull = 1,
-    kEmpty = 5,
-    kRotFull = 9,
-    kEReady = 11,
-    kProjFull = 13,
-    kTmemEmpty = 15,
-    kNormReady = 17
+    kFull = 1,       // [4] input stage landed
+    kEmpty = 5,      // [4] input stage consumed (rotation + both norm warps)
+    kRotFull = 9,    // [4] rotation accumulator ready
+    kEReady = 13,    // [4] codes written; keys: residual in TMEM; values: accumulator free
+    kNormReady = 17, // [4] squared row norms of the slot's tile
+    kPartReady = 21, // [4] half-1 residual norms handed to half 0
+    kProjFull = 25,  // [2] projection accumulator ready (and its residual operand consumed)
+    kAccFree = 27    // [2] projection accumulator read
 };
 
 // Code of y against ascending boundaries b[0..2^BETA-2] (#{k : b[k] < y}) by a binary
@@ -92,41 +109,17 @@ __device__ __forceinline__ void bucket_bits(float y, const float (&b)[16], bool 
     }
 }
 
-template <int N>
-__device__ __forceinline__ uint32_t umux(const uint32_t *v, uint32_t idx) {
-    if constexpr (N == 1) {
-        return v[0];
-    } else {
-        const uint32_t lo = umux<N / 2>(v, idx);
-        const uint32_t hi = umux<N / 2>(v + N / 2, idx);
-        return (idx & (N / 2)) ? hi : lo;
-    }
-}
-
-// v[idx] for a register array, as a tree of selects.
-template <int N>
-__device__ __forceinline__ float mux(const float *v, uint32_t idx) {
-    if constexpr (N == 1) {
-        return v[0];
-    } else {
-        const float lo = mux<N / 2>(v, idx);
-        const float hi = mux<N / 2>(v + N / 2, idx);
-        return (idx & (N / 2)) ? hi : lo;
-    }
-}
-
 template <int D, bool IS_KEY, int BETA>
 __global__ void __launch_bounds__(kThreads, 1)
     compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, Prepared P, int64_t n,
                        uint32_t *__restrict__ codes, uint32_t *__restrict__ signs, uint16_t *__restrict__ norm,
                        uint16_t *__restrict__ rnorm, int32_t *__restrict__ dev_status) {
-    constexpr int KB = D / 64;
     constexpr int KSTEPS = D / 16;
     constexpr int CHUNKS = D / 32;
     constexpr uint32_t XSTAGE = kTileRows * D * 2;
     const int m = IS_KEY ? P.m : 0;
     const TcSmem L = tc_smem_layout(D, m, IS_KEY);
-    const int NST = L.nst;
+    const int NST = L.nst, NRS = L.nrs;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -135,8 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *cen_s = bnd_s + kMaxLevels;
     uint32_t *tmem_s = (uint32_t *)(cen_s + kMaxLevels);
     volatile int *abort_s = (volatile int *)(tmem_s + 1);
-    float *norm_s = (float *)(sm + L.misc + 256);  // [2 slots][128 rows] squared norms
-    uint32_t *cbit_s = (uint32_t *)(sm + L.misc + 256 + 1024);  // centroid fp16 hi/lo bits
+    float *norm_s = (float *)(sm + L.misc + kMiscNorm);    // [slot][row] squared norms
+    float *ee_s = (float *)(sm + L.misc + kMiscEe);        // [slot][row] half residual norms
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
@@ -147,25 +140,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars[kFull + s], 1);
             mbar_init(&bars[kEmpty + s], 3);  // MMA commit + the two norm warps
+            mbar_init(&bars[kRotFull + s], 1);
+            mbar_init(&bars[kEReady + s], 8);
+            mbar_init(&bars[kNormReady + s], 2);
+            mbar_init(&bars[kPartReady + s], 4);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[kRotFull + s], 1);
-            mbar_init(&bars[kEReady + s], 4);
             mbar_init(&bars[kProjFull + s], 1);
-            mbar_init(&bars[kTmemEmpty + s], 4);
-            mbar_init(&bars[kNormReady + s], 2);
+            mbar_init(&bars[kAccFree + s], 8);
         }
         *abort_s = 0;
         fence_mbar_init();
     }
     if (threadIdx.x < kMaxLevels) {
         bnd_s[threadIdx.x] = IS_KEY ? P.cb->kb[threadIdx.x] : P.cb->vb[threadIdx.x];
-        const float c = IS_KEY ? P.cb->kc[threadIdx.x] : P.cb->vc[threadIdx.x];
-        cen_s[threadIdx.x] = c;
-        const float cs = c * (float)(1 << kCScaleLog2);
-        const __half h = __float2half_rn(cs);
-        const __half lo = __float2half_rn(cs - __half2float(h));
-        cbit_s[threadIdx.x] = ((uint32_t)__half_as_ushort(h) << 16) | (uint32_t)__half_as_ushort(lo);
+        cen_s[threadIdx.x] = IS_KEY ? P.cb->kc[threadIdx.x] : P.cb->vc[threadIdx.x];
     }
     if (warp == 0) {
         tmem_alloc(tmem_s, 512);
@@ -180,10 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmap);
-            const uint32_t rbytes = 2u * (IS_KEY ? D + m : D) * D * 2;
+            const uint32_t rbytes = 2u * D * D * 2;
             const uint32_t sbytes = IS_KEY ? 2u * m * D * 2 : 0u;
             mbar_arrive_expect_tx(&bars[kOpnd], rbytes + sbytes);
-            bulk_load(sm + L.R, IS_KEY ? P.RSsw : P.Rsw, rbytes, &bars[kOpnd]);
+            bulk_load(sm + L.R, P.Rsw, rbytes, &bars[kOpnd]);
             if (IS_KEY) bulk_load(sm + L.S, P.Ssw, sbytes, &bars[kOpnd]);
             int issued = 0;
             for (int i = 0; i < my_tiles; ++i) {
@@ -193,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *dst = sm + L.X + stage * XSTAGE;
                 mbar_arrive_expect_tx(&bars[kFull + stage], XSTAGE);
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
+                for (int kb = 0; kb < D / 64; ++kb)
                     tma_load_2d(dst + kb * (kTileRows * 128), &tmap, &bars[kFull + stage], kb * 64,
                                 (int)(tile * kTileRows));
                 ++issued;
@@ -207,21 +196,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const int rowsB = IS_KEY ? D + m : D;
-            const uint32_t idesc_rot = idesc_f16_f32(128, rowsB);
+            const uint32_t idesc_rot = idesc_f16_f32(128, D);
             const uint32_t idesc_prj = idesc_f16_f32(128, m > 0 ? m : 16);
             const uint32_t sR = smem_u32(sm + L.R), sS = smem_u32(sm + L.S), sX = smem_u32(sm + L.X);
             bool ok = mbar_wait(&bars[kOpnd], 0, abort_s);
-            auto projection = [&](int j) -> bool {
-                const int slot = j & 1;
-                if (!mbar_wait(&bars[kEReady + slot], (j >> 1) & 1, abort_s)) return false;
+            // rotation of tile i into accumulator slot i % NRS, once the slot's previous tile has
+            // released it (keys: its residual was consumed by the projection; values: its codes
+            // are out)
+            auto rotation = [&](int i) -> bool {
+                const int rs = i % NRS, stage = i % NST;
+                if (i >= NRS) {
+                    const bool w = IS_KEY ? mbar_wait(&bars[kProjFull + ((i - NRS) & 1)], ((i - NRS) >> 1) & 1, abort_s)
+                                          : mbar_wait(&bars[kEReady + rs], ((i / NRS) - 1) & 1, abort_s);
+                    if (!w) return false;
+                }
+                if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) return false;
                 tc_fence_after();
-                const uint32_t acc = tmem + slot * 256 + D + m;
+                const uint32_t acc = tmem + rs * D;
+                const uint32_t xbase = sX + stage * XSTAGE;
+                uint32_t first = 0;
+#pragma unroll
+                for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                    for (int k = 0; k < KSTEPS; ++k) {
+                        const uint32_t aoff = (uint32_t)(k >> 2) * (kTileRows * 128) + (k & 3) * 32;
+                        const uint32_t boff = (uint32_t)pass * (D * D * 2) + (uint32_t)(k >> 2) * (D * 128) + (k & 3) * 32;
+                        mma_ss(acc, sdesc_sw128(xbase + aoff), sdesc_sw128(sR + boff), idesc_rot, first);
+                        first = 1;
+                    }
+                mma_commit(&bars[kEmpty + stage]);
+                mma_commit(&bars[kRotFull + rs]);
+                return true;
+            };
+            // projection of tile j's residual (hi | lo in its rotation slot) into accumulator j & 1
+            auto projection = [&](int j) -> bool {
+                const int rs = j % NRS, pa = j & 1;
+                if (!mbar_wait(&bars[kEReady + rs], (j / NRS) & 1, abort_s)) return false;
+                if (j >= 2 && !mbar_wait(&bars[kAccFree + pa], ((j >> 1) - 1) & 1, abort_s)) return false;
+                tc_fence_after();
+                const uint32_t acc = tmem + NRS * D + pa * m;
                 const uint32_t sbytes = (uint32_t)m * D * 2;
                 uint32_t first = 0;
 #pragma unroll 1
                 for (int k = 0; k < KSTEPS; ++k) {
-                    const uint32_t a_hi = tmem + slot * 256 + 32 * (k >> 1) + 8 * (k & 1);
+                    const uint32_t a_hi = tmem + rs * D + 32 * (k >> 1) + 8 * (k & 1);
                     const uint32_t a_lo = a_hi + 16;
                     const uint32_t boff = (uint32_t)(k >> 2) * m * 128 + (k & 3) * 32;
                     const uint64_t b_hi = sdesc_sw128(sS + boff);
@@ -231,98 +249,129 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ts(acc, a_hi, b_lo, idesc_prj, 1);
                     mma_ts(acc, a_lo, b_hi, idesc_prj, 1);
                 }
-                mma_commit(&bars[kProjFull + slot]);
+                mma_commit(&bars[kProjFull + pa]);
                 return true;
             };
-            auto rotation = [&](int i) -> bool {
-                const int slot = i & 1, stage = i % NST;
-                if (i >= 2 && !mbar_wait(&bars[kTmemEmpty + slot], ((i >> 1) - 1) & 1, abort_s)) return false;
-                if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) return false;
-                tc_fence_after();
-                const uint32_t acc = tmem + slot * 256;
-                const uint32_t xbase = sX + stage * XSTAGE;
-                uint32_t first = 0;
-#pragma unroll
-                for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                    for (int k = 0; k < KSTEPS; ++k) {
-                        const uint32_t aoff = (uint32_t)(k >> 2) * (kTileRows * 128) + (k & 3) * 32;
-                        const uint32_t boff = (uint32_t)pass * (rowsB * D * 2) + (uint32_t)(k >> 2) * (rowsB * 128) +
-                                              (k & 3) * 32;
-                        mma_ss(acc, sdesc_sw128(xbase + aoff), sdesc_sw128(sR + boff), idesc_rot, first);
-                        first = 1;
-                    }
-                mma_commit(&bars[kEmpty + stage]);
-                mma_commit(&bars[kRotFull + slot]);
-                return true;
-            };
-            // Two tiles in flight (one per TMEM slot); the projection of tile j goes out as soon
-            // as its residual is ready, before the rotation that reuses tile j's slot.
-            if (ok && my_tiles > 0) ok = rotation(0);
-            if (ok && my_tiles > 1) ok = rotation(1);
-            for (int j = 0; ok && j < my_tiles; ++j) {
-                if (IS_KEY && !projection(j)) break;
-                if (j + 2 < my_tiles && !rotation(j + 2)) break;
+            if (IS_KEY) {
+                // rotations run NRS - 1 tiles ahead of the projections
+                for (int i = 0; ok && i < NRS - 1 && i < my_tiles; ++i) ok = rotation(i);
+                for (int j = 0; ok && j < my_tiles; ++j) {
+                    if (!projection(j)) break;
+                    if (j + NRS - 1 < my_tiles && !rotation(j + NRS - 1)) break;
+                }
+            } else {
+                for (int i = 0; ok && i < my_tiles; ++i) ok = rotation(i);
             }
         }
     } else if (warp < kNormWarp0) {
         // ------------------------------------------------------------ epilogue
+        // Every tile goes to all eight warps: warp (q, h) takes rows 32q..32q+31 (its TMEM lane
+        // quarter) and half h of the coordinates and of the projections.  Keys run the code step
+        // of tile i, then the sign step of tile i - 1, so the projection of tile i - 1 executes
+        // on the tensor cores while tile i is being coded.
         const int ew = warp - kEpiWarp0;   // 0..7
-        const int wg = ew >> 2;            // which half of the tiles / TMEM
+        const int h = ew >> 2;             // which half of the columns
         const int q = warp & 3;            // TMEM subpartition this warp may access
         const int row = 32 * q + lane;     // vector within the tile
-        const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)wg * 256;
+        const uint32_t lanes = (uint32_t)(32 * q) << 16;
+        constexpr int CH = CHUNKS / 2;     // 32-coordinate chunks per warp
         constexpr int wpv = BETA * CHUNKS;
+        const int spk = m >> 5;
         float bnd_r[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) bnd_r[k] = bnd_s[k];
-        for (int i = wg; i < my_tiles; i += 2) {
+        // The key codebook is symmetric (c[H + k] = -c[H - 1 - k] exactly, middle boundary 0), so
+        // with two or four levels a key coordinate's centroid follows from its sign bit and
+        // magnitude bit; the scaled centroids stay in registers.
+        constexpr int H = (IS_KEY && BETA <= 2) ? (1 << BETA) / 2 : 1;
+        float cpos[H], cneg[H];
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+            cpos[k] = cen_s[H + k] * (float)(1 << kEScaleLog2);
+            cneg[k] = -cpos[k];
+        }
+
+        // codes of tile i; keys also leave 2^14 (y - c) as fp16 hi | lo in the slot's columns
+        auto code_step = [&](int i) -> bool {
+            const int rs = i % NRS;
+            const uint32_t ph = (uint32_t)(i / NRS) & 1;
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
             const int64_t v = tile * kTileRows + row;
             const bool valid = v < n;
-            if (!mbar_wait(&bars[kNormReady + wg], (i >> 1) & 1, abort_s)) break;
-            if (!mbar_wait(&bars[kRotFull + wg], (i >> 1) & 1, abort_s)) break;
+            if (!mbar_wait(&bars[kNormReady + rs], ph, abort_s)) return false;
+            if (!mbar_wait(&bars[kRotFull + rs], ph, abort_s)) return false;
             tc_fence_after();
-            const float nx = sqrtf(norm_s[wg * kTileRows + row]);
+            const float nx = sqrtf(norm_s[rs * kTileRows + row]);
             // the accumulator holds 2^8 R x; y = R x / ||x||
             const float inv = nx > 0.f ? (1.0f / (float)(1 << kRScaleLog2)) / nx : 0.f;
-            float ee = 0.f;
-            uint32_t r[32];
+            const float inve = inv * (float)(1 << kEScaleLog2);
+            // two- and four-level keys compare the accumulator itself against boundaries scaled by
+            // 2^8 ||x||; a zero vector compares its zero accumulator against the unscaled ones
+            float bsc[16];
+            if constexpr (IS_KEY && BETA <= 2) {
+                const float sc = nx > 0.f ? nx * (float)(1 << kRScaleLog2) : 1.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) bsc[k] = bnd_r[k] * sc;
+            }
+            float ee = 0.f;  // sum of (2^14 (y - c))^2 over this warp's coordinates
+            const uint32_t tl = tmem + lanes + rs * D;
             uint32_t *dst = codes + v * wpv;
-            // chunks of 32 coordinates; the loop stays rolled so the unrolled body fits the
-            // instruction cache, and each chunk's code words go straight to global memory
+            uint32_t r[32];
+            // the loop stays rolled so the unrolled body fits the instruction cache
 #pragma unroll 1
-            for (int c = 0; c < CHUNKS; ++c) {
+            for (int c = h * CH; c < h * CH + CH; ++c) {
                 tmem_ld32(tl + 32 * c, r);
                 tmem_ld_wait();
                 uint32_t wp[4] = {0u, 0u, 0u, 0u};
-                uint32_t hp[16], lp[16];
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
-                    const float y = __uint_as_float(r[l]) * inv;
                     bool t[4];
-                    bucket_bits<BETA>(y, bnd_r, t);
-                    uint32_t idx = 0;
+                    if constexpr (IS_KEY && BETA <= 2) {
+                        const float a = __uint_as_float(r[l]);
+                        bucket_bits<BETA>(a, bsc, t);
 #pragma unroll
-                    for (int p = 0; p < BETA; ++p) {
-                        if (t[p]) wp[p] |= 1u << l;
-                        idx |= (t[p] ? 1u : 0u) << p;
-                    }
-                    if (IS_KEY) {
-                        // centroid and its fp16 hi/lo bit pattern from shared-memory tables
-                        const float e = y - cen_s[idx];
-                        ee = fmaf(e, e, ee);
-                        const uint32_t cb = cbit_s[idx];
-                        if (l & 1) {
-                            hp[l >> 1] = __byte_perm(hp[l >> 1], cb, 0x7632);
-                            lp[l >> 1] = __byte_perm(lp[l >> 1], cb, 0x5410);
+                        for (int p = 0; p < BETA; ++p)
+                            if (t[p]) wp[p] |= 1u << l;
+                        // t[BETA-1] is the sign; the magnitude bit is set where t[0] agrees with it
+                        const bool pos = t[BETA - 1];
+                        float cs;
+                        if constexpr (H == 1) {
+                            cs = pos ? cpos[0] : cneg[0];
                         } else {
-                            hp[l >> 1] = cb;
-                            lp[l >> 1] = cb;
+                            const bool m0 = t[0] == pos;
+                            cs = pos ? (m0 ? cpos[1] : cpos[0]) : (m0 ? cneg[1] : cneg[0]);
+                        }
+                        const float es = fmaf(a, inve, -cs);
+                        ee = fmaf(es, es, ee);
+                        r[l] = __float_as_uint(es);
+                    } else {
+                        const float y = __uint_as_float(r[l]) * inv;
+                        bucket_bits<BETA>(y, bnd_r, t);
+                        uint32_t idx = 0;
+#pragma unroll
+                        for (int p = 0; p < BETA; ++p) {
+                            if (t[p]) wp[p] |= 1u << l;
+                            idx |= (t[p] ? 1u : 0u) << p;
+                        }
+                        if constexpr (IS_KEY) {
+                            const float es = (y - cen_s[idx]) * (float)(1 << kEScaleLog2);
+                            ee = fmaf(es, es, ee);
+                            r[l] = __float_as_uint(es);
                         }
                     }
                 }
-                if (IS_KEY) {
+                if constexpr (IS_KEY) {
+                    // fp16 hi | lo split of the scaled residual, two coordinates per column
+                    uint32_t hp[16], lp[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float ea = __uint_as_float(r[2 * k]), eb = __uint_as_float(r[2 * k + 1]);
+                        const __half2 hh = __floats2half2_rn(ea, eb);
+                        const float2 hf = __half22float2(hh);
+                        const __half2 ll = __floats2half2_rn(ea - hf.x, eb - hf.y);
+                        hp[k] = *(const uint32_t *)&hh;
+                        lp[k] = *(const uint32_t *)&ll;
+                    }
                     tmem_st16(tl + 32 * c, hp);
                     tmem_st16(tl + 32 * c + 16, lp);
                 }
@@ -331,51 +380,77 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int p = 0; p < BETA; ++p) dst[c * BETA + p] = wp[p];
                 }
             }
-            if (IS_KEY) tmem_st_wait();
+            if constexpr (IS_KEY) {
+                tmem_st_wait();
+                // half 1 hands its part of ||y - c||^2 to half 0; ee_s[rs] is next written NRS
+                // tiles on, after half 0 has released this slot
+                if (h == 1) {
+                    ee_s[rs * kTileRows + row] = ee;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[kPartReady + rs]);
+                } else {
+                    if (!mbar_wait(&bars[kPartReady + rs], ph, abort_s)) return false;
+                    const float ss = (ee + ee_s[rs * kTileRows + row]) * (1.0f / (float)(1 << (2 * kEScaleLog2)));
+                    if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ss));
+                }
+            }
+            if (valid && h == 0) norm[v] = f32_to_f16_bits(nx);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(IS_KEY ? &bars[kEReady + wg] : &bars[kTmemEmpty + wg]);
-            if (valid) norm[v] = f32_to_f16_bits(nx);
-            if (IS_KEY) {
-                if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
-                if (!mbar_wait(&bars[kProjFull + wg], (i >> 1) & 1, abort_s)) break;
-                tc_fence_after();
-                // p = S u - S' c[idx]: S u from the rotation accumulator (2^8 S x), S' c from the
-                // projection accumulator (2^(kCScaleLog2 + kSScaleLog2) S' c)
-                const int spk = m >> 5;
-                const float pun = 1.0f / (float)(1 << (kCScaleLog2 + kSScaleLog2));
+            if (lane == 0) mbar_arrive(&bars[kEReady + rs]);
+            return true;
+        };
+
+        // QJL signs of tile j from its projection accumulator (2^18 S' (y - c))
+        auto sign_step = [&](int j) -> bool {
+            const int pa = j & 1;
+            const int64_t tile = blockIdx.x + (int64_t)j * gridDim.x;
+            const int64_t v = tile * kTileRows + row;
+            const bool valid = v < n;
+            if (!mbar_wait(&bars[kProjFull + pa], (j >> 1) & 1, abort_s)) return false;
+            tc_fence_after();
+            const uint32_t ta = tmem + lanes + NRS * D + pa * m;
+            uint32_t r[32];
 #pragma unroll 1
-                for (int g = 0; g < spk; ++g) {
-                    uint32_t r2[32];
-                    tmem_ld32(tl + D + 32 * g, r);
-                    tmem_ld32(tl + D + m + 32 * g, r2);
-                    tmem_ld_wait();
-                    uint32_t sw = 0;
+            for (int g = h; g < spk; g += 2) {
+                tmem_ld32(ta + 32 * g, r);
+                tmem_ld_wait();
+                uint32_t sw = 0;
 #pragma unroll
-                    for (int l = 0; l < 32; ++l) {
-                        const float pv = fmaf(__uint_as_float(r[l]), inv, -__uint_as_float(r2[l]) * pun);
-                        sw |= (uint32_t)(pv >= 0.f) << l;
-                    }
-                    if (valid) signs[v * spk + g] = sw;
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[kTmemEmpty + wg]);
+                for (int l = 0; l < 32; ++l) sw |= (uint32_t)(__uint_as_float(r[l]) >= 0.f) << l;
+                if (valid) signs[v * spk + g] = sw;
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kAccFree + pa]);
+            return true;
+        };
+
+        if (IS_KEY) {
+            bool ok = true;
+            for (int i = 0; ok && i < my_tiles; ++i) {
+                ok = code_step(i);
+                if (ok && i >= 1) ok = sign_step(i - 1);
+            }
+            if (ok && my_tiles > 0) sign_step(my_tiles - 1);
+        } else {
+            for (int i = 0; i < my_tiles; ++i)
+                if (!code_step(i)) break;
         }
     } else {
         // ------------------------------------------------------------ row norms
         // ||x||^2 of every row of the fp16 input tile, read from the swizzled stage in
-        // shared memory (exact fp16 inputs, fp32 sums); two warps, 64 rows each.
+        // shared memory (exact fp16 inputs, fp32 sums); two warps, 64 rows each.  Slot rs of
+        // norm_s is rewritten once the code step of the tile NRS earlier has read it.
         const int nw = warp - kNormWarp0;
         for (int i = 0; i < my_tiles; ++i) {
-            const int slot = i & 1, stage = i % NST;
-            if (i >= 2 && !mbar_wait(&bars[kTmemEmpty + slot], ((i >> 1) - 1) & 1, abort_s)) break;
+            const int rs = i % NRS, stage = i % NST;
+            if (i >= NRS && !mbar_wait(&bars[kEReady + rs], ((i / NRS) - 1) & 1, abort_s)) break;
             if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) break;
             const uint8_t *xs = sm + L.X + stage * XSTAGE;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = nw * 64 + h * 32 + lane;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = nw * 64 + hh * 32 + lane;
                 float ss = 0.f;
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
@@ -389,11 +464,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ss = fmaf(f.y, f.y, ss);
                     }
                 }
-                norm_s[slot * kTileRows + r] = ss;
+                norm_s[rs * kTileRows + r] = ss;
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bars[kNormReady + slot]);
+                mbar_arrive(&bars[kNormReady + rs]);
                 mbar_arrive(&bars[kEmpty + stage]);
             }
         }
@@ -454,8 +529,8 @@ cudaError_t launch_tc(const Prepared &P, const void *x, int64_t n, uint32_t *cod
 bool compress_tc_supported(const Prepared &P, bool is_key, bool x_f16) {
     if (!x_f16) return false;
     if (P.d != 128 && P.d != 64) return false;
-    // keys keep [R x | S x] and the projection in one 256-column TMEM slot
-    if (is_key && (P.m < 32 || P.m % 32 || P.d + 2 * P.m > 256)) return false;
+    // keys need two rotation accumulators beside the two projection accumulators
+    if (is_key && (P.m < 32 || P.m % 32 || P.m > 256 || tc_rotation_slots(P.d, P.m, true) < 2)) return false;
     return true;
 }
 
