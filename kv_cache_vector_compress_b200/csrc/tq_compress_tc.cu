@@ -87,25 +87,21 @@ enum BarIdx {
     kAccFree = 27    // [2] projection accumulator read
 };
 
-// Code of y against ascending boundaries b[0..2^BETA-2] (#{k : b[k] < y}) by a binary
-// search whose thresholds are selected from registers; t[p] receives bit p of the code.
+// Magnitude digits of u = |y| against the HL - 1 = 2^(BETA-1) - 1 positive boundaries e[] of a
+// symmetric codebook (binary search, thresholds selected from registers): mb[j] receives bit j
+// of m = #{k : e[k] < u}.  The code of y is then HL + m for y > 0 and HL - 1 - m otherwise, so its
+// low bits are m's bits, complemented on the negative side, and its top bit is the sign.
 template <int BETA>
-__device__ __forceinline__ void bucket_bits(float y, const float (&b)[16], bool (&t)[4]) {
-    if constexpr (BETA == 1) {
-        t[0] = y > b[0];
-    } else if constexpr (BETA == 2) {
-        t[1] = y > b[1];
-        t[0] = y > (t[1] ? b[2] : b[0]);
+__device__ __forceinline__ void magnitude_bits(float u, const float *e, bool (&mb)[3]) {
+    if constexpr (BETA == 2) {
+        mb[0] = u > e[0];
     } else if constexpr (BETA == 3) {
-        t[2] = y > b[3];
-        t[1] = y > (t[2] ? b[5] : b[1]);
-        t[0] = y > (t[2] ? (t[1] ? b[6] : b[4]) : (t[1] ? b[2] : b[0]));
-    } else {
-        t[3] = y > b[7];
-        t[2] = y > (t[3] ? b[11] : b[3]);
-        t[1] = y > (t[3] ? (t[2] ? b[13] : b[9]) : (t[2] ? b[5] : b[1]));
-        t[0] = y > (t[3] ? (t[2] ? (t[1] ? b[14] : b[12]) : (t[1] ? b[10] : b[8]))
-                         : (t[2] ? (t[1] ? b[6] : b[4]) : (t[1] ? b[2] : b[0])));
+        mb[1] = u > e[1];
+        mb[0] = u > (mb[1] ? e[2] : e[0]);
+    } else if constexpr (BETA == 4) {
+        mb[2] = u > e[3];
+        mb[1] = u > (mb[2] ? e[5] : e[1]);
+        mb[0] = u > (mb[2] ? (mb[1] ? e[6] : e[4]) : (mb[1] ? e[2] : e[0]));
     }
 }
 
@@ -277,19 +273,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int CH = CHUNKS / 2;     // 32-coordinate chunks per warp
         constexpr int wpv = BETA * CHUNKS;
         const int spk = m >> 5;
-        float bnd_r[16];
+        // Both codebooks are symmetric (c[HL + k] = -c[HL - 1 - k] exactly, middle boundary 0), so a
+        // coordinate is coded from its sign and the magnitude digits of |y| against the HL - 1
+        // positive boundaries; a key's centroid is sign(y) cmag[m] and (y - c)^2 = (|y| - cmag[m])^2.
+        constexpr int HL = 1 << (BETA - 1);
+        float edge[HL > 1 ? HL - 1 : 1];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) bnd_r[k] = bnd_s[k];
-        // The key codebook is symmetric (c[H + k] = -c[H - 1 - k] exactly, middle boundary 0), so
-        // with two or four levels a key coordinate's centroid follows from its sign bit and
-        // magnitude bit; the scaled centroids stay in registers.
-        constexpr int H = (IS_KEY && BETA <= 2) ? (1 << BETA) / 2 : 1;
-        float cpos[H], cneg[H];
+        for (int k = 0; k < HL - 1; ++k) edge[k] = bnd_s[HL + k];
+        float cmag[HL];  // 2^14 |c| (keys)
 #pragma unroll
-        for (int k = 0; k < H; ++k) {
-            cpos[k] = cen_s[H + k] * (float)(1 << kEScaleLog2);
-            cneg[k] = -cpos[k];
-        }
+        for (int k = 0; k < HL; ++k) cmag[k] = cen_s[HL + k] * (float)(1 << kEScaleLog2);
 
         // codes of tile i; keys also leave 2^14 (y - c) as fp16 hi | lo in the slot's columns
         auto code_step = [&](int i) -> bool {
@@ -305,14 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the accumulator holds 2^8 R x; y = R x / ||x||
             const float inv = nx > 0.f ? (1.0f / (float)(1 << kRScaleLog2)) / nx : 0.f;
             const float inve = inv * (float)(1 << kEScaleLog2);
-            // two- and four-level keys compare the accumulator itself against boundaries scaled by
-            // 2^8 ||x||; a zero vector compares its zero accumulator against the unscaled ones
-            float bsc[16];
-            if constexpr (IS_KEY && BETA <= 2) {
-                const float sc = nx > 0.f ? nx * (float)(1 << kRScaleLog2) : 1.f;
+            // the accumulator itself is compared against boundaries scaled by 2^8 ||x||; a zero
+            // vector compares its zero accumulator against the unscaled ones (y = 0)
+            const float sc = nx > 0.f ? nx * (float)(1 << kRScaleLog2) : 1.f;
+            float ep[HL > 1 ? HL - 1 : 1];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) bsc[k] = bnd_r[k] * sc;
-            }
+            for (int k = 0; k < HL - 1; ++k) ep[k] = edge[k] * sc;
             float ee = 0.f;  // sum of (2^14 (y - c))^2 over this warp's coordinates
             const uint32_t tl = tmem + lanes + rs * D;
             uint32_t *dst = codes + v * wpv;
@@ -325,39 +316,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t wp[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
-                    bool t[4];
-                    if constexpr (IS_KEY && BETA <= 2) {
-                        const float a = __uint_as_float(r[l]);
-                        bucket_bits<BETA>(a, bsc, t);
+                    const float a = __uint_as_float(r[l]);
+                    const bool pos = a > 0.f;
+                    bool mb[3];
+                    magnitude_bits<BETA>(fabsf(a), ep, mb);
+                    if (pos) wp[BETA - 1] |= 1u << l;
 #pragma unroll
-                        for (int p = 0; p < BETA; ++p)
-                            if (t[p]) wp[p] |= 1u << l;
-                        // t[BETA-1] is the sign; the magnitude bit is set where t[0] agrees with it
-                        const bool pos = t[BETA - 1];
-                        float cs;
-                        if constexpr (H == 1) {
-                            cs = pos ? cpos[0] : cneg[0];
-                        } else {
-                            const bool m0 = t[0] == pos;
-                            cs = pos ? (m0 ? cpos[1] : cpos[0]) : (m0 ? cneg[1] : cneg[0]);
-                        }
-                        const float es = fmaf(a, inve, -cs);
-                        ee = fmaf(es, es, ee);
-                        r[l] = __float_as_uint(es);
-                    } else {
-                        const float y = __uint_as_float(r[l]) * inv;
-                        bucket_bits<BETA>(y, bnd_r, t);
-                        uint32_t idx = 0;
-#pragma unroll
-                        for (int p = 0; p < BETA; ++p) {
-                            if (t[p]) wp[p] |= 1u << l;
-                            idx |= (t[p] ? 1u : 0u) << p;
-                        }
-                        if constexpr (IS_KEY) {
-                            const float es = (y - cen_s[idx]) * (float)(1 << kEScaleLog2);
-                            ee = fmaf(es, es, ee);
-                            r[l] = __float_as_uint(es);
-                        }
+                    for (int j = 0; j < BETA - 1; ++j)
+                        if (mb[j] == pos) wp[j] |= 1u << l;
+                    if constexpr (IS_KEY) {
+                        float cm;
+                        if constexpr (HL == 1) cm = cmag[0];
+                        else if constexpr (HL == 2) cm = mb[0] ? cmag[1] : cmag[0];
+                        else cm = mb[1] ? (mb[0] ? cmag[3] : cmag[2]) : (mb[0] ? cmag[1] : cmag[0]);
+                        const float em = fmaf(fabsf(a), inve, -cm);  // 2^14 (|y| - |c|)
+                        ee = fmaf(em, em, ee);
+                        r[l] = __float_as_uint(em) ^ (pos ? 0u : 0x80000000u);  // 2^14 (y - c)
                     }
                 }
                 if constexpr (IS_KEY) {
