@@ -233,7 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t acc = tmem + NRS * D + pa * m;
                 const uint32_t sbytes = (uint32_t)m * D * 2;
                 uint32_t first = 0;
-#pragma unroll 1
+                // unrolled: a single thread issues the MMAs, and loop overhead between issues
+                // would starve the tensor cores (N = 64 MMAs take about 45 cycles each)
+#pragma unroll
                 for (int k = 0; k < KSTEPS; ++k) {
                     const uint32_t a_hi = tmem + rs * D + 32 * (k >> 1) + 8 * (k & 1);
                     const uint32_t a_lo = a_hi + 16;
@@ -304,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float ep[HL > 1 ? HL - 1 : 1];
 #pragma unroll
             for (int k = 0; k < HL - 1; ++k) ep[k] = edge[k] * sc;
-            float ee = 0.f;  // sum of (2^14 (y - c))^2 over this warp's coordinates
+            float2 ee2 = make_float2(0.f, 0.f);  // sums of (2^14 (y - c))^2 over even / odd coordinates
             const uint32_t tl = tmem + lanes + rs * D;
             uint32_t *dst = codes + v * wpv;
             uint32_t r[32];
@@ -314,40 +316,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tl + 32 * c, r);
                 tmem_ld_wait();
                 uint32_t wp[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-                for (int l = 0; l < 32; ++l) {
-                    const float a = __uint_as_float(r[l]);
-                    const bool pos = a > 0.f;
-                    bool mb[3];
-                    magnitude_bits<BETA>(fabsf(a), ep, mb);
-                    if (pos) wp[BETA - 1] |= 1u << l;
-#pragma unroll
-                    for (int j = 0; j < BETA - 1; ++j)
-                        if (mb[j] == pos) wp[j] |= 1u << l;
-                    if constexpr (IS_KEY) {
-                        float cm;
-                        if constexpr (HL == 1) cm = cmag[0];
-                        else if constexpr (HL == 2) cm = mb[0] ? cmag[1] : cmag[0];
-                        else cm = mb[1] ? (mb[0] ? cmag[3] : cmag[2]) : (mb[0] ? cmag[1] : cmag[0]);
-                        const float em = fmaf(fabsf(a), inve, -cm);  // 2^14 (|y| - |c|)
-                        ee = fmaf(em, em, ee);
-                        r[l] = __float_as_uint(em) ^ (pos ? 0u : 0x80000000u);  // 2^14 (y - c)
-                    }
-                }
                 if constexpr (IS_KEY) {
-                    // fp16 hi | lo split of the scaled residual, two coordinates per column
+                    // coordinate pairs: codes, then 2^14 (y - c) and its fp16 hi | lo split with
+                    // packed two-wide fp32 arithmetic (one column holds the pair)
                     uint32_t hp[16], lp[16];
+                    const float2 inve2 = make_float2(inve, inve);
+                    const float2 mone2 = make_float2(-1.f, -1.f);
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        const float ea = __uint_as_float(r[2 * k]), eb = __uint_as_float(r[2 * k + 1]);
-                        const __half2 hh = __floats2half2_rn(ea, eb);
-                        const float2 hf = __half22float2(hh);
-                        const __half2 ll = __floats2half2_rn(ea - hf.x, eb - hf.y);
+                        float ncs[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int l = 2 * k + u;
+                            const float a = __uint_as_float(r[l]);
+                            const bool pos = a > 0.f;
+                            bool mb[3];
+                            magnitude_bits<BETA>(fabsf(a), ep, mb);
+                            if (pos) wp[BETA - 1] |= 1u << l;
+#pragma unroll
+                            for (int j = 0; j < BETA - 1; ++j)
+                                if (mb[j] == pos) wp[j] |= 1u << l;
+                            float cm;
+                            if constexpr (HL == 1) cm = cmag[0];
+                            else if constexpr (HL == 2) cm = mb[0] ? cmag[1] : cmag[0];
+                            else cm = mb[1] ? (mb[0] ? cmag[3] : cmag[2]) : (mb[0] ? cmag[1] : cmag[0]);
+                            ncs[u] = __uint_as_float(__float_as_uint(cm) ^ (pos ? 0x80000000u : 0u));  // -2^14 c
+                        }
+                        const float2 a2 = make_float2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+                        const float2 e2 = __ffma2_rn(a2, inve2, make_float2(ncs[0], ncs[1]));  // 2^14 (y - c)
+                        ee2 = __ffma2_rn(e2, e2, ee2);
+                        const __half2 hh = __floats2half2_rn(e2.x, e2.y);
+                        const float2 d2 = __ffma2_rn(__half22float2(hh), mone2, e2);
+                        const __half2 ll = __floats2half2_rn(d2.x, d2.y);
                         hp[k] = *(const uint32_t *)&hh;
                         lp[k] = *(const uint32_t *)&ll;
                     }
                     tmem_st16(tl + 32 * c, hp);
                     tmem_st16(tl + 32 * c + 16, lp);
+                } else {
+#pragma unroll
+                    for (int l = 0; l < 32; ++l) {
+                        const float a = __uint_as_float(r[l]);
+                        const bool pos = a > 0.f;
+                        bool mb[3];
+                        magnitude_bits<BETA>(fabsf(a), ep, mb);
+                        if (pos) wp[BETA - 1] |= 1u << l;
+#pragma unroll
+                        for (int j = 0; j < BETA - 1; ++j)
+                            if (mb[j] == pos) wp[j] |= 1u << l;
+                    }
                 }
                 if (valid) {
 #pragma unroll
@@ -358,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 // half 1 hands its part of ||y - c||^2 to half 0; ee_s[rs] is next written NRS
                 // tiles on, after half 0 has released this slot
+                const float ee = ee2.x + ee2.y;
                 if (h == 1) {
                     ee_s[rs * kTileRows + row] = ee;
                     __syncwarp();
