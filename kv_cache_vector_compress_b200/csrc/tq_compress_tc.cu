@@ -28,9 +28,14 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileRows = 128;
-constexpr int kThreads = 384;  // 12 warps
 constexpr int kEpiWarp0 = 2;   // warps 2..9: epilogue (two groups of four)
-constexpr int kNormWarp0 = 10; // warps 10..11: row norms of the input tiles
+constexpr int kNormWarp0 = 10; // warps 10..: row norms of the input tiles
+// Row-norm warps: four, one per SM sub-partition, so the code step's sub-partitions carry equal
+// work; two for the register-heavy eight-level keys and sixteen-level values.
+template <bool IS_KEY, int BETA>
+constexpr int tc_norm_warps() { return (IS_KEY ? BETA == 3 : BETA == 4) ? 2 : 4; }
+template <bool IS_KEY, int BETA>
+constexpr int tc_threads() { return 32 * (kNormWarp0 + tc_norm_warps<IS_KEY, BETA>()); }
 constexpr int kEScaleLog2 = 14;  // residual scale before the fp16 hi/lo split
 
 struct TcSmem {
@@ -106,7 +111,7 @@ __device__ __forceinline__ void magnitude_bits(float u, const float *e, bool (&m
 }
 
 template <int D, bool IS_KEY, int BETA>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
     compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, Prepared P, int64_t n,
                        uint32_t *__restrict__ codes, uint32_t *__restrict__ signs, uint16_t *__restrict__ norm,
                        uint16_t *__restrict__ rnorm, int32_t *__restrict__ dev_status) {
@@ -116,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = IS_KEY ? P.m : 0;
     const TcSmem L = tc_smem_layout(D, m, IS_KEY);
     const int NST = L.nst, NRS = L.nrs;
+    constexpr int NW = tc_norm_warps<IS_KEY, BETA>();
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -135,10 +141,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars[kOpnd], 1);
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars[kFull + s], 1);
-            mbar_init(&bars[kEmpty + s], 3);  // MMA commit + the two norm warps
+            mbar_init(&bars[kEmpty + s], 1 + NW);  // MMA commit + the norm warps
             mbar_init(&bars[kRotFull + s], 1);
             mbar_init(&bars[kEReady + s], 8);
-            mbar_init(&bars[kNormReady + s], 2);
+            mbar_init(&bars[kNormReady + s], NW);
             mbar_init(&bars[kPartReady + s], 4);
         }
         for (int s = 0; s < 2; ++s) {
@@ -432,7 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ row norms
         // ||x||^2 of every row of the fp16 input tile, read from the swizzled stage in
-        // shared memory (exact fp16 inputs, fp32 sums); two warps, 64 rows each.  Slot rs of
+        // shared memory (exact fp16 inputs, fp32 sums of even and odd coordinates); NW warps,
+        // 128 / NW rows each.  Slot rs of
         // norm_s is rewritten once the code step of the tile NRS earlier has read it.
         const int nw = warp - kNormWarp0;
         for (int i = 0; i < my_tiles; ++i) {
@@ -441,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) break;
             const uint8_t *xs = sm + L.X + stage * XSTAGE;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = nw * 64 + hh * 32 + lane;
-                float ss = 0.f;
+            for (int hh = 0; hh < 4 / NW; ++hh) {
+                const int r = nw * (kTileRows / NW) + hh * 32 + lane;
+                float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
                     const int kb = c >> 3, cc = c & 7;
@@ -452,10 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = __half22float2(*(const __half2 *)&u[e]);
-                        ss = fmaf(f.x, f.x, ss);
-                        ss = fmaf(f.y, f.y, ss);
+                        ss2 = __ffma2_rn(f, f, ss2);
                     }
                 }
+                const float ss = ss2.x + ss2.y;
                 norm_s[rs * kTileRows + r] = ss;
             }
             __syncwarp();
@@ -511,7 +518,7 @@ cudaError_t launch_tc(const Prepared &P, const void *x, int64_t n, uint32_t *cod
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    compress_tc_kernel<D, IS_KEY, BETA><<<grid, kThreads, smem, s>>>(map, P, n, codes, signs, norm, rnorm,
+    compress_tc_kernel<D, IS_KEY, BETA><<<grid, tc_threads<IS_KEY, BETA>(), smem, s>>>(map, P, n, codes, signs, norm, rnorm,
                                                                    dev_status);
     return cudaGetLastError();
 }
