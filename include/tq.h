@@ -182,6 +182,33 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
                     int32_t *dev_status, tq_stream_t stream);
 
 /*
+ * tq_append_attend -- one decode step on caches with spare capacity: append the new token of
+ * every (batch, KV head), then attend over the cache including it.
+ * The append is TurboQuantProd.compress / TurboQuantMSE.quantize of the new key / value and the
+ * attention is that of tq_attend, as the cache wrapper does them token by token
+ * ("turboquant-pytorch", nav.superapi.store, 核心 API: TurboQuantKVCache with append_key,
+ * append_value, attention_scores; "TurboQuant: онлайн-квантование векторов без калибровки",
+ * ai-manual.ru, "Где TurboQuant выстреливает, а где нет?": keys and values compressed during
+ * generation).  The compression runs inside the attention kernel, in the CTA whose context range
+ * holds slot t, so the step launches no separate compress kernel.
+ *   q            : device fp32 [B, Hq, Nq, dim]
+ *   k_new, v_new : device [B, Hkv, dim] of dtype (TQ_F16 or TQ_F32), 16-byte aligned
+ *   t            : the slot the new token takes, 0 <= t < t_cap; slots 0 .. t-1 hold the cache
+ *   t_cap        : cache capacity: every array below holds B * Hkv * t_cap records, record
+ *                  (b * Hkv + h) * t_cap + s for slot s of (b, h), in the layouts of
+ *                  tq_compress_keys / tq_compress_values; slot t is overwritten
+ *   scale, out   : as tq_attend; the attention covers slots 0 .. t (t + 1 tokens)
+ *   scratch      : tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, t + 1) bytes
+ * Returns TQ_ERR_UNSUPPORTED for shapes outside the tensor-core attention kernel (dim 64, 128 or
+ * 256, proj_dim = dim / 2, 2-4 bit keys), and the errors of tq_attend.
+ */
+tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new, const void *v_new,
+                           tq_dtype dtype, int B, int Hq, int Hkv, int Nq, int64_t t, int64_t t_cap,
+                           uint32_t *kcodes, uint32_t *ksigns, uint16_t *knorm, uint16_t *krnorm,
+                           uint32_t *vcodes, uint16_t *vnorm, float scale, float *out, void *scratch,
+                           size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream);
+
+/*
  * tq_selftest_wait_timeout -- exercises the device-side failure path of every kernel.
  * (The pages have no counterpart: this is a diagnostic of the library.)
  * Every wait of the kernels on another warp or on a copy is bounded; when one runs out, the

@@ -47,11 +47,13 @@ ScoreProblem make_problem(int B, int Hq, int Hkv, int Nq, int64_t T, const float
                           const uint32_t *ksigns, const uint16_t *knorm, const uint16_t *krnorm,
                           const uint32_t *vcodes, const uint16_t *vnorm) {
     ScoreProblem sp;
+    memset(&sp, 0, sizeof(sp));
     sp.B = B;
     sp.Hq = Hq;
     sp.Hkv = Hkv;
     sp.Nq = Nq;
     sp.T = T;
+    sp.Ts = T;
     sp.q = q;
     sp.kcodes = kcodes;
     sp.ksigns = ksigns;
@@ -253,6 +255,50 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
             e = launch_attend(P, sp, qprep, scale, partials, plan.splits, out, s);
         }
     }
+    return from_cuda(e);
+}
+
+tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new, const void *v_new,
+                           tq_dtype dtype, int B, int Hq, int Hkv, int Nq, int64_t t, int64_t t_cap,
+                           uint32_t *kcodes, uint32_t *ksigns, uint16_t *knorm, uint16_t *krnorm,
+                           uint32_t *vcodes, uint16_t *vnorm, float scale, float *out, void *scratch,
+                           size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
+    (void)dev_status;
+    tq_status st = check_params(p, true);
+    if (st != TQ_OK) return st;
+    if (t < 0 || t_cap < 1 || t >= t_cap) return TQ_ERR_INVALID_ARG;
+    if (dtype != TQ_F16 && dtype != TQ_F32) return TQ_ERR_INVALID_ARG;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return TQ_ERR_INVALID_ARG;
+    // the checks of tq_attend, over the whole cache extent
+    st = check_problem(p, B, Hq, Hkv, Nq, t_cap, q, kcodes, ksigns, knorm, krnorm);
+    if (st != TQ_OK) return st;
+    if (!vcodes || !vnorm || !out || !aligned16(vcodes) || !aligned16(vnorm) || !aligned16(out))
+        return TQ_ERR_INVALID_ARG;
+    if (!(scale == scale)) return TQ_ERR_INVALID_ARG;  // NaN
+    if (!scratch || !aligned16(scratch)) return TQ_ERR_INVALID_ARG;
+    if (scratch_bytes < tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, t + 1)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, t + 1, q, kcodes, ksigns, knorm, krnorm, vcodes, vnorm);
+    sp.Ts = t_cap;
+    sp.knew = k_new;
+    sp.vnew = v_new;
+    sp.new_f16 = dtype == TQ_F16;
+    sp.tnew = t;
+    sp.kcodes_w = kcodes;
+    sp.ksigns_w = ksigns;
+    sp.knorm_w = knorm;
+    sp.krnorm_w = krnorm;
+    sp.vcodes_w = vcodes;
+    sp.vnorm_w = vnorm;
+    const AttendPlan plan = plan_attend(P, sp);
+    if (!plan.mma) return TQ_ERR_UNSUPPORTED;
+    if (scale <= 0.f) scale = 1.0f / sqrtf((float)p->dim);
+    cudaStream_t s = (cudaStream_t)stream;
+    float *qprep = (float *)scratch;
+    float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
+    cudaError_t e = launch_qprep(P, sp, qprep, s);
+    if (e == cudaSuccess) e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
+    if (e == cudaSuccess) e = launch_attend_combine(P, sp, partials, plan.splits, out, s);
     return from_cuda(e);
 }
 

@@ -23,6 +23,7 @@
 #include <math.h>
 
 #include "tq_common.cuh"
+#include "tq_compress_warp.cuh"
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -232,6 +233,36 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     uint16_t *ptile = (uint16_t *)(smem + L.ptile) + warp * (2 * kRowsPerCta * 16);
     uint16_t *ptile_lo = ptile + kRowsPerCta * 16;
     for (int e = lane; e < 2 * kRowsPerCta * 16; e += 32) ptile[e] = 0;
+    // ---- decode-step append: a CTA whose token range holds record tnew first compresses the
+    // slice's new key (warp 0) and value (warp 1) into the caches, then reads it back with the
+    // rest of its range.  Every CTA of the slice that holds the record (one per row group)
+    // writes the same bytes.  Scratch: the per-warp stage area, not yet in use.
+    if constexpr (ATTEND) {
+        if (sp.knew != nullptr && sp.tnew >= t0 && sp.tnew < t1 && warp < 2) {
+            float *us = (float *)(smem + L.stage) + warp * D;
+            const int64_t rec = sl * sp.Ts + sp.tnew;
+            if (warp == 0) {
+                if (sp.new_f16)
+                    compress_vector_warp<G32, true, true>(P, sp.knew, sl, P.cb->kb, P.cb->kc, us, lane,
+                                                          sp.kcodes_w + rec * KWPT, sp.ksigns_w + rec * SW,
+                                                          sp.knorm_w + rec, sp.krnorm_w + rec);
+                else
+                    compress_vector_warp<G32, true, false>(P, sp.knew, sl, P.cb->kb, P.cb->kc, us, lane,
+                                                           sp.kcodes_w + rec * KWPT, sp.ksigns_w + rec * SW,
+                                                           sp.knorm_w + rec, sp.krnorm_w + rec);
+            } else {
+                if (sp.new_f16)
+                    compress_vector_warp<G32, false, true>(P, sp.vnew, sl, P.cb->vb, P.cb->vc, us, lane,
+                                                           sp.vcodes_w + rec * VWPT, nullptr, sp.vnorm_w + rec,
+                                                           nullptr);
+                else
+                    compress_vector_warp<G32, false, false>(P, sp.vnew, sl, P.cb->vb, P.cb->vc, us, lane,
+                                                            sp.vcodes_w + rec * VWPT, nullptr, sp.vnorm_w + rec,
+                                                            nullptr);
+            }
+            __threadfence();
+        }
+    }
     __syncthreads();
 
     // ---- B fragments (queries) in registers
@@ -274,8 +305,8 @@ __global__ void __launch_bounds__(kThreadsMma) decode_mma_kernel(Prepared P, Sco
     const int64_t wt1 = min(t1, wt0 + wlen);
     const int NST = L.nst;
     uint8_t *wstage = smem + L.stage + (size_t)warp * NST * L.stage_bytes;
-    const int64_t rec_base = sl * sp.T;
-    const int64_t nrec = (int64_t)sp.B * sp.Hkv * sp.T;
+    const int64_t rec_base = sl * sp.Ts;
+    const int64_t nrec = (int64_t)sp.B * sp.Hkv * sp.Ts;
     // fp16 norms of records [rec0, rec0 + ntok): 4-byte words from the even index below rec0; an
     // odd last element that would take its word past the end of the arrays is copied directly
     auto stage_norms = [&](uint16_t *dst, const uint16_t *src, int64_t rec0, int ntok) {

@@ -139,12 +139,21 @@ cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool 
 
 struct ScoreProblem {
     int B, Hq, Hkv, Nq;
-    int64_t T;
+    int64_t T;   // tokens scored / attended per (batch, KV head)
+    int64_t Ts;  // record stride of the caches: slice s holds records s * Ts .. s * Ts + T - 1
     const float *q;
     const uint32_t *kcodes, *ksigns;
     const uint16_t *knorm, *krnorm;
     const uint32_t *vcodes;
     const uint16_t *vnorm;
+    // decode-step append: when knew is set, the attention kernel first compresses row s of knew
+    // and vnew ([B * Hkv, d], fp16 or fp32) into record s * Ts + tnew of the caches below (the
+    // same arrays as the read-only pointers above)
+    const void *knew, *vnew;
+    int new_f16;
+    int64_t tnew;
+    uint32_t *kcodes_w, *ksigns_w, *vcodes_w;
+    uint16_t *knorm_w, *krnorm_w, *vnorm_w;
 };
 
 size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp);

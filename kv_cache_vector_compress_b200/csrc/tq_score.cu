@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kTile) scores_kernel(Prepared P, ScoreProblem 
     const int rows = (sp.Hq / sp.Hkv) * sp.Nq;
     const int64_t t = (int64_t)blockIdx.x * kTile + threadIdx.x;
     const bool valid = t < sp.T;
-    const int64_t rec = sl * sp.T + t;
+    const int64_t rec = sl * sp.Ts + t;
     const float gamma = sqrtf(1.5707963267948966f) / (float)m;
     const int wpk = P.kbeta * (d >> 5), spk = m >> 5;
     float kn = 0.f, rn = 0.f;
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kTile) attend_kernel(Prepared P, ScoreProblem 
                 for (int r = 0; r < RM; ++r) acc[r] = acc2[r] = 0.f;
                 float kn = 0.f, rn = 0.f;
                 if (valid) {
-                    const int64_t rec = sl * sp.T + t;
+                    const int64_t rec = sl * sp.Ts + t;
                     kn = f16_bits_to_f32(sp.knorm[rec]);
                     rn = f16_bits_to_f32(sp.krnorm[rec]);
                     key_dots<RM>(P, kcen, qs, rch, sp.kcodes + rec * wpk, sp.ksigns + rec * spk, acc, acc2);
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kTile) attend_kernel(Prepared P, ScoreProblem 
                 }
             const int ntok = (int)min((int64_t)kTile, t1 - tb);
             for (int tt = 0; tt < ntok; ++tt) {
-                const int64_t rec = sl * sp.T + tb + tt;
+                const int64_t rec = sl * sp.Ts + tb + tt;
                 const float vn = f16_bits_to_f32(sp.vnorm[rec]);
                 const uint32_t *vw = sp.vcodes + rec * vwpv;
 #pragma unroll

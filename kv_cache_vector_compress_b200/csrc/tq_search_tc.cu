@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     const int sl = unit / g.nrb;
     const int my_tiles = (int)((g.nkt - cidx + g.kc - 1) / g.kc);
     const int total = my_tiles * NKB;
-    const int64_t rec_base = (int64_t)sl * sp.T;
+    const int64_t rec_base = (int64_t)sl * sp.Ts;
     const int E = uexp[unit * 2], eA = uexp[unit * 2 + 1];
 
     if (threadIdx.x == 0) {

@@ -56,6 +56,9 @@ _lib.tq_scores_scratch_bytes.argtypes = [_PP, _I, _I, _I, _I, _I64, _I]
 _lib.tq_scores_scratch_bytes.restype = _SZ
 _lib.tq_scores.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P, _P]
 _lib.tq_scores.restype = _I
+_lib.tq_append_attend.argtypes = [_PP, _P, _P, _P, _I, _I, _I, _I, _I, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                  ctypes.c_float, _P, _P, _SZ, _P, _P]
+_lib.tq_append_attend.restype = _I
 _lib.tq_attend_scratch_bytes.argtypes = [_PP, _I, _I, _I, _I, _I64]
 _lib.tq_attend_scratch_bytes.restype = _SZ
 _lib.tq_attend.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
@@ -72,7 +75,8 @@ TQ_STATIC_SCRATCH_BYTES = 16 << 20
 
 EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_workspace_bytes", "tq_prepare",
            "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores",
-           "tq_attend_scratch_bytes", "tq_attend", "tq_selftest_wait_timeout", "tq_attend_static"]
+           "tq_attend_scratch_bytes", "tq_attend", "tq_append_attend", "tq_selftest_wait_timeout",
+           "tq_attend_static"]
 
 
 class TQError(RuntimeError):
@@ -231,6 +235,30 @@ def tq_attend(p: Params, q: torch.Tensor, keys, values, Hkv: int, T: int, scale:
     _check(_lib.tq_attend(p.ref, _ptr(q), B, Hq, Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr),
                           _ptr(vc), _ptr(vn), float(scale), _ptr(out), _ptr(scratch), scratch.numel(),
                           _ptr(dev_status), _stream()), "tq_attend")
+    return out
+
+
+def tq_append_attend(p: Params, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, keys, values,
+                     Hkv: int, t: int, t_cap: int, scale: float = 0.0, out=None, scratch=None, dev_status=None):
+    """One decode step: compress the new token of every (batch, KV head) (k_new, v_new: [B, Hkv, dim],
+    fp16 or fp32) into slot t of the caches (keys / values as returned by the compress calls, holding
+    B * Hkv * t_cap records), then attend over slots 0 .. t.  Returns out [B, Hq, Nq, dim] fp32."""
+    B, Hq, Nq, d = q.shape
+    kc, ks, kn, kr = keys
+    vc, vn = values
+    if k_new.dtype != v_new.dtype or k_new.dtype not in (torch.float16, torch.float32):
+        raise ValueError("k_new and v_new must both be float16 or both float32")
+    dt = 0 if k_new.dtype == torch.float16 else 1
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.float32, device=dev)
+    if scratch is None:
+        scratch = torch.empty(max(tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, t + 1), 16), dtype=torch.uint8,
+                              device=dev)
+    _check(_lib.tq_append_attend(p.ref, _ptr(q), _ptr(k_new), _ptr(v_new), dt, B, Hq, Hkv, Nq, t, t_cap,
+                                 _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr), _ptr(vc), _ptr(vn), float(scale),
+                                 _ptr(out), _ptr(scratch), scratch.numel(), _ptr(dev_status), _stream()),
+           "tq_append_attend")
     return out
 
 

@@ -325,3 +325,71 @@ def test_end_to_end_workload1(tq):
             & (as_u16(kt[2]) == k["norm"]) & (as_u16(kt[3]) == k["rnorm"]))
     assert same.mean() > 0.999
     check_close(s[0, 0][:, torch.from_numpy(same).cuda()], ora_s[0, 0][:, same], "end-to-end scores")
+
+
+# ------------------------------------------------------- decode-step append + attend
+
+@pytest.mark.parametrize("cfg", [
+    dict(d=128, m=64, bits=3, B=2, Hkv=2, G=4, Nq=1, t=1000, cap=1100, f16=True),   # GQA decode step
+    dict(d=64, m=32, bits=2, B=1, Hkv=3, G=1, Nq=2, t=0, cap=5, f16=False),         # empty cache, fp32 rows
+    dict(d=256, m=128, bits=4, B=1, Hkv=1, G=8, Nq=1, t=4094, cap=4095, f16=True),  # last slot, wide head
+    dict(d=128, m=64, bits=2, B=1, Hkv=1, G=16, Nq=1, t=333, cap=400, f16=True),    # two row groups
+])
+def test_append_attend(tq, cfg):
+    """tq_append_attend writes the oracle's records for the new token into slot t, leaves every other
+    slot alone, and attends over slots 0..t exactly as the oracle does over that cache."""
+    import torch
+    c = cfg
+    d, m, bits, B, Hkv, t, cap = c["d"], c["m"], c["bits"], c["B"], c["Hkv"], c["t"], c["cap"]
+    Hq, nsl = Hkv * c["G"], B * Hkv
+    seed = 500 + d + t
+    R, S = synth.rotation(d, seed), synth.gaussian(m, d, seed + 1)
+    dt = np.float16 if c["f16"] else np.float32
+    # every slot of the cache holds a valid record, so reading past slot t would change the output
+    K = synth.gaussian(nsl * cap, d, seed + 2).astype(np.float16)
+    V = synth.gaussian(nsl * cap, d, seed + 3).astype(np.float16)
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    v = oracle.compress(V, R, None, bits, is_key=False)
+    k_new = synth.gaussian(nsl, d, seed + 4).astype(dt)
+    v_new = synth.gaussian(nsl, d, seed + 5).astype(dt)
+    q = synth.gaussian(B * Hq * c["Nq"], d, seed + 6).reshape(B, Hq, c["Nq"], d)
+    p = _params(tq, R, S, bits, m)
+    kk, vv = _to_dev(k, v)
+    out = tq.tq_append_attend(p, torch.from_numpy(q).cuda(), torch.from_numpy(k_new).cuda(),
+                              torch.from_numpy(v_new).cuda(), kk, vv, Hkv, t, cap)
+    torch.cuda.synchronize()
+
+    def slots(a):
+        a = a.cpu().numpy() if hasattr(a, "cpu") else a
+        return a.reshape(nsl, cap, -1)
+
+    g = {n: slots(x) for n, x in zip(("kc", "ks", "kn", "kr"), kk)}
+    g.update({n: slots(x) for n, x in zip(("vc", "vn"), vv)})
+    # the new records against the oracle's compression of the new rows
+    kb, vb = bits - 1, bits
+    ok_ = oracle.compress(k_new, R, S, bits, is_key=True, want_y=True, want_p=True)
+    ov_ = oracle.compress(v_new, R, None, bits, is_key=False, want_y=True)
+    rows = check_codes(g["kc"][:, t].view(np.uint32), ok_["codes"], ok_["y32"], oracle.codebook_f32(d, kb)[0], d, kb,
+                       what="appended key codes")
+    check_signs(g["ks"][:, t].view(np.uint32), ok_["signs"], ok_["p32"], m, exempt_rows=rows, what="appended signs")
+    check_f16_close(g["kn"][:, t].view(np.uint16).ravel(), ok_["norm"], what="appended key norm")
+    check_f16_close(g["kr"][:, t].view(np.uint16).ravel(), ok_["rnorm"], exempt_rows=rows, what="appended rnorm")
+    check_codes(g["vc"][:, t].view(np.uint32), ov_["codes"], ov_["y32"], oracle.codebook_f32(d, vb)[0], d, vb,
+                what="appended value codes")
+    check_f16_close(g["vn"][:, t].view(np.uint16).ravel(), ov_["norm"], what="appended value norm")
+    # every other slot untouched
+    other = np.ones(cap, bool)
+    other[t] = False
+    for name, ref in (("kc", k["codes"]), ("ks", k["signs"]), ("kn", k["norm"]), ("kr", k["rnorm"]),
+                      ("vc", v["codes"]), ("vn", v["norm"])):
+        gv = g[name][:, other].reshape(-1).view(np.uint16 if name in ("kn", "kr", "vn") else np.uint32)
+        rv = ref.reshape(nsl, cap, -1)[:, other].reshape(-1)
+        assert np.array_equal(gv, rv), f"slot other than t changed in {name}"
+    # attention over slots 0..t of the cache as the GPU left it
+    def upto(a, dtype):
+        r = np.ascontiguousarray(a[:, : t + 1]).view(dtype).reshape(nsl * (t + 1), -1)
+        return r[:, 0] if r.shape[1] == 1 else r
+    ora = oracle.attend(q, R, S, bits, B, Hq, Hkv, c["Nq"], t + 1, upto(g["kc"], np.uint32), upto(g["ks"], np.uint32),
+                        upto(g["kn"], np.uint16), upto(g["kr"], np.uint16), upto(g["vc"], np.uint32),
+                        upto(g["vn"], np.uint16))
+    check_close(out, ora, "append + attend")
