@@ -472,6 +472,71 @@ def run_workload(args):
         r["frac_tensor"] = r["tflops_mma"] / pk["bf16_tflops"] if pk.get("bf16_tflops") else None
         out.append(r)
         name = f"vector search: {N} x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
+    elif wl == 6:
+        # one decode step on the decode-attention shape: append the new token of every (batch, KV
+        # head) into slot t of a cache of capacity T, then attend over slots 0..t
+        d, m, bits, B, Hq, Hkv, T = 128, 64, 3, 32, 32, 8, 32768
+        B = args.batch if args.batch > 0 else B
+        t, ns = T - 1, B * Hkv
+        n = ns * T
+        R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
+        S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
+        p = tq.Params(d, bits, m, R, S)
+        keys = tq.tq_compress_keys(p, synth.torch_normal_f16((n, d), s["keys"]))
+        vals = tq.tq_compress_values(p, synth.torch_normal_f16((n, d), s["values"]))
+        kn = synth.torch_normal_f16((B, Hkv, d), s["scales"] + 1)
+        vn = synth.torch_normal_f16((B, Hkv, d), s["scales"] + 2)
+        Q = synth.torch_normal_f32((B, Hq, 1, d), s["queries"])
+        o = torch.empty((B, Hq, 1, d), dtype=torch.float32, device="cuda")
+        scr = torch.empty(tq.tq_attend_scratch_bytes(p, B, Hq, Hkv, 1, T), dtype=torch.uint8, device="cuda")
+        kb, vb = (bits - 1) * d // 8 + m // 8 + 4, bits * d // 8 + 2
+        nbytes = ns * (t + 1) * (kb + vb) + ns * 2 * d * 2
+        ms = timed(lambda: tq.tq_append_attend(p, Q, kn, vn, keys, vals, Hkv, t, T, out=o, scratch=scr))
+        out.append(rec("append_attend", ms, ns * (t + 1), "keys", nbytes))
+        # the same step unfused: compress the B * Hkv new rows, then attend over the cache
+        nk = tq.tq_compress_keys(p, kn.view(ns, d))
+        nv = tq.tq_compress_values(p, vn.view(ns, d))
+
+        def unfused():
+            tq.tq_compress_keys(p, kn.view(ns, d), *nk)
+            tq.tq_compress_values(p, vn.view(ns, d), *nv)
+            tq.tq_attend(p, Q, keys, vals, Hkv, T, out=o, scratch=scr)
+        ms = timed(unfused)
+        out.append(rec("compress_new_then_attend", ms, ns * (t + 1), "keys", nbytes))
+        name = (f"decode step: B{B} Hq32/Hkv8 d128 3-bit, append the new token into slot {t} of a "
+                f"{T}-slot cache, attend over {t + 1} tokens")
+    elif wl == 7:
+        # attention quality of the compressed cache on synthetic Qwen2.5-3B-shaped decode inputs
+        # (36 layers x 2 KV heads as the batch, 16 query heads, 8K context, one query per head),
+        # two input recipes: "gaussian" (keys, values, queries N(0,1): the coordinate model the
+        # method is built on) and "key_outliers" (keys N(0,1) x lognormal(0,1) per (layer, KV
+        # head, channel), as real key caches have outlier channels; values, queries N(0,1))
+        from kv_cache_vector_compress_b200 import quality
+        d, m, L, Hkv, Hq, T = 128, 64, 36, 2, 16, 8192
+        R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
+        S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
+        sc = torch.from_numpy(np.exp(np.random.Generator(np.random.PCG64(s["scales"])).standard_normal(
+            (L, Hkv, 1, d))).astype(np.float32)).cuda()
+        V = synth.torch_normal_f16((L, Hkv, T, d), s["values"])
+        Q = synth.torch_normal_f32((L, Hq, 1, d), s["queries"])
+        res = {}
+        for recipe in ("gaussian", "key_outliers"):
+            K = synth.torch_normal_f16((L, Hkv, T, d), s["keys"])
+            if recipe == "key_outliers":
+                K = (K.float() * sc).half()
+            res[recipe] = []
+            for bits in (2, 3, 4):
+                p = tq.Params(d, bits, m, R, S)
+                keys = tq.tq_compress_keys(p, K.view(-1, d))
+                vals = tq.tq_compress_values(p, V.view(-1, d))
+                res[recipe].append({"bits": bits, **quality.attention_quality(p, Q, K, V, keys, vals)})
+        print(json.dumps({"workload": wl, "name": "attention quality, synthetic Qwen2.5-3B-shaped decode: "
+                          "36 layers x 2 KV heads, 16 query heads, T8192, d128 (means over 576 query rows)",
+                          "quality": res,
+                          "pages_qwen_validation": {"note": "real activations, not comparable",
+                                                    "cosine": {"4": 0.999, "3": 0.995, "2": 0.988},
+                                                    "top1": {"4": 0.87, "3": 0.82, "2": 0.66}}}), flush=True)
+        return 0
     else:
         raise SystemExit("unknown workload")
     print(json.dumps({"workload": wl, "name": name, "ops": out, "peak_hbm_gbs": pk["hbm_gbs"]}), flush=True)
@@ -489,7 +554,8 @@ def main():
     ap.add_argument("--db", type=int, default=0,
                     help="database vectors of the vector-search workload (default 1,000,000; smaller for profiling)")
     ap.add_argument("--workload", type=int, default=3,
-                    help="3 (default) prints the headline line; 1, 2, 4, 5 print secondary per-op measurements")
+                    help="3 (default) prints the headline line; 1, 2, 4, 5, 6 print secondary per-op "
+                         "measurements, 7 the attention quality of the compressed cache")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
