@@ -156,6 +156,22 @@ def test_argument_errors_return_before_any_launch(lib):
     assert att(10, out=None) == 1
     assert att(10, sb=16) == 1
     assert att(10, scale=float("nan")) == 1
+    # decode-step append: slot outside the cache, bad dtype, missing or misaligned new rows
+    L.tq_append_attend.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                   ctypes.c_void_p, ctypes.c_void_p]
+    app = lambda t, cap, kn=fake, dt=0, sb=1 << 40: L.tq_append_attend(
+        P(good), fake, kn, fake, dt, 1, 4, 2, 1, t, cap, fake, fake, fake, fake, fake, fake, 0.0, fake, fake,
+        sb, None, None)
+    assert app(10, 10) == 1        # slot t must be below the capacity
+    assert app(-1, 10) == 1
+    assert app(3, 10, dt=5) == 1   # dtype
+    assert app(3, 10, kn=None) == 1
+    assert app(3, 10, kn=fake + 8) == 1
+    assert app(3, 10, sb=16) == 1  # scratch too small
 
 
 def test_scratch_size_helpers(lib):
