@@ -190,7 +190,7 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
  * append_value, attention_scores; "TurboQuant: онлайн-квантование векторов без калибровки",
  * ai-manual.ru, "Где TurboQuant выстреливает, а где нет?": keys and values compressed during
  * generation).  The compression runs inside the attention kernel, in the CTA whose context range
- * holds slot t, so the step launches no separate compress kernel.
+ * holds slot t, so the step launches no separate compress kernel (tensor-core attention shapes).
  *   q            : device fp32 [B, Hq, Nq, dim]
  *   k_new, v_new : device [B, Hkv, dim] of dtype (TQ_F16 or TQ_F32), 16-byte aligned
  *   t            : the slot the new token takes, 0 <= t < t_cap; slots 0 .. t-1 hold the cache
@@ -199,8 +199,9 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
  *                  tq_compress_keys / tq_compress_values; slot t is overwritten
  *   scale, out   : as tq_attend; the attention covers slots 0 .. t (t + 1 tokens)
  *   scratch      : tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, t + 1) bytes
- * Returns TQ_ERR_UNSUPPORTED for shapes outside the tensor-core attention kernel (dim 64, 128 or
- * 256, proj_dim = dim / 2, 2-4 bit keys), and the errors of tq_attend.
+ * For shapes outside the tensor-core attention kernel (dim 64, 128 or 256 with proj_dim = dim / 2
+ * and 2-4 bit keys) the append is a small kernel of its own, launched before the attention.
+ * Returns the errors of tq_attend.
  */
 tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new, const void *v_new,
                            tq_dtype dtype, int B, int Hq, int Hkv, int Nq, int64_t t, int64_t t_cap,

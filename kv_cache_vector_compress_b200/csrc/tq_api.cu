@@ -291,14 +291,22 @@ tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new
     sp.vcodes_w = vcodes;
     sp.vnorm_w = vnorm;
     const AttendPlan plan = plan_attend(P, sp);
-    if (!plan.mma) return TQ_ERR_UNSUPPORTED;
     if (scale <= 0.f) scale = 1.0f / sqrtf((float)p->dim);
     cudaStream_t s = (cudaStream_t)stream;
     float *qprep = (float *)scratch;
     float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
     cudaError_t e = launch_qprep(P, sp, qprep, s);
-    if (e == cudaSuccess) e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
-    if (e == cudaSuccess) e = launch_attend_combine(P, sp, partials, plan.splits, out, s);
+    if (plan.mma) {
+        // the append runs inside the attention kernel
+        if (e == cudaSuccess) e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
+        if (e == cudaSuccess) e = launch_attend_combine(P, sp, partials, plan.splits, out, s);
+    } else {
+        // other shapes: the append kernel, then the CUDA-core attention over the strided cache
+        if (e == cudaSuccess) e = launch_append(P, sp, s);
+        ScoreProblem rd = sp;
+        rd.knew = rd.vnew = nullptr;
+        if (e == cudaSuccess) e = launch_attend(P, rd, qprep, scale, partials, plan.splits, out, s);
+    }
     return from_cuda(e);
 }
 

@@ -35,6 +35,39 @@ __global__ void __launch_bounds__(kWarps * 32)
                                                  IS_KEY ? rnorm + v : nullptr);
 }
 
+// Decode-step append for shapes outside the tensor-core attention kernel: warp 2s compresses the
+// new key of slice s, warp 2s+1 its new value, into record s * Ts + tnew of the caches.
+template <int NPL, bool X_F16>
+__global__ void __launch_bounds__(kWarps * 32) append_kernel(Prepared P, ScoreProblem sp) {
+    constexpr int D = NPL * 32;
+    __shared__ float vec[kWarps][D];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t nsl = (int64_t)sp.B * sp.Hkv;
+    const int64_t job = (int64_t)blockIdx.x * kWarps + warp;
+    if (job >= 2 * nsl) return;
+    const int64_t sl = job >> 1;
+    const int64_t rec = sl * sp.Ts + sp.tnew;
+    if ((job & 1) == 0) {
+        const int mpl = P.m >> 5;
+        compress_vector_warp<NPL, true, X_F16>(P, sp.knew, sl, P.cb->kb, P.cb->kc, vec[warp], lane,
+                                               sp.kcodes_w + rec * (P.kbeta * NPL), sp.ksigns_w + rec * mpl,
+                                               sp.knorm_w + rec, sp.krnorm_w + rec);
+    } else {
+        compress_vector_warp<NPL, false, X_F16>(P, sp.vnew, sl, P.cb->vb, P.cb->vc, vec[warp], lane,
+                                                sp.vcodes_w + rec * (P.vbeta * NPL), nullptr, sp.vnorm_w + rec,
+                                                nullptr);
+    }
+}
+
+template <int NPL>
+cudaError_t launch_append_npl(const Prepared &P, const ScoreProblem &sp, cudaStream_t s) {
+    const int64_t jobs = 2 * (int64_t)sp.B * sp.Hkv;
+    const unsigned blocks = (unsigned)((jobs + kWarps - 1) / kWarps);
+    if (sp.new_f16) append_kernel<NPL, true><<<blocks, kWarps * 32, 0, s>>>(P, sp);
+    else append_kernel<NPL, false><<<blocks, kWarps * 32, 0, s>>>(P, sp);
+    return cudaGetLastError();
+}
+
 template <int NPL>
 cudaError_t launch_npl(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
                        uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
@@ -56,6 +89,18 @@ cudaError_t launch_npl(const Prepared &P, bool is_key, const void *x, bool x_f16
 }
 
 }  // namespace
+
+cudaError_t launch_append(const Prepared &P, const ScoreProblem &sp, cudaStream_t s) {
+    switch (P.d) {
+        case 32: return launch_append_npl<1>(P, sp, s);
+        case 64: return launch_append_npl<2>(P, sp, s);
+        case 128: return launch_append_npl<4>(P, sp, s);
+        case 256: return launch_append_npl<8>(P, sp, s);
+        case 512: return launch_append_npl<16>(P, sp, s);
+        case 1024: return launch_append_npl<32>(P, sp, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
                             uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,

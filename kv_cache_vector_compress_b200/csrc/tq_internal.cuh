@@ -156,6 +156,8 @@ struct ScoreProblem {
     uint16_t *knorm_w, *krnorm_w, *vnorm_w;
 };
 
+// Compress the new key / value of every slice into record s * Ts + tnew (sp.knew, sp.vnew set).
+cudaError_t launch_append(const Prepared &P, const ScoreProblem &sp, cudaStream_t s);
 size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp);
 int attend_splits(const ScoreProblem &sp);
 size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int splits);
