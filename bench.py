@@ -530,9 +530,18 @@ def run_workload(args):
                 keys = tq.tq_compress_keys(p, K.view(-1, d))
                 vals = tq.tq_compress_values(p, V.view(-1, d))
                 res[recipe].append({"bits": bits, **quality.attention_quality(p, Q, K, V, keys, vals)})
+        # proj_dim sweep at 3 bits on the gaussian recipe: the QJL term's variance falls as 1/m
+        K = synth.torch_normal_f16((L, Hkv, T, d), s["keys"])
+        sweep = []
+        for mm in (32, 64, 128):
+            Sm = torch.from_numpy(synth.gaussian(mm, d, s["S"] + mm)).cuda()
+            p = tq.Params(d, 3, mm, R, Sm)
+            keys = tq.tq_compress_keys(p, K.view(-1, d))
+            vals = tq.tq_compress_values(p, V.view(-1, d))
+            sweep.append({"proj_dim": mm, **quality.attention_quality(p, Q, K, V, keys, vals)})
         print(json.dumps({"workload": wl, "name": "attention quality, synthetic Qwen2.5-3B-shaped decode: "
                           "36 layers x 2 KV heads, 16 query heads, T8192, d128 (means over 576 query rows)",
-                          "quality": res,
+                          "quality": res, "proj_dim_sweep_3bit_gaussian": sweep,
                           "pages_qwen_validation": {"note": "real activations, not comparable",
                                                     "cosine": {"4": 0.999, "3": 0.995, "2": 0.988},
                                                     "top1": {"4": 0.87, "3": 0.82, "2": 0.66}}}), flush=True)
