@@ -539,9 +539,17 @@ def run_workload(args):
             keys = tq.tq_compress_keys(p, K.view(-1, d))
             vals = tq.tq_compress_values(p, V.view(-1, d))
             sweep.append({"proj_dim": mm, **quality.attention_quality(p, Q, K, V, keys, vals)})
+        # ablation: MSE-only keys (b MSE bits, no QJL) against the two-stage keys, scores only
+        mse = []
+        for b in (2, 3):
+            pv = tq.Params(d, b, m, R, S)
+            codes, norm = tq.tq_compress_values(pv, K.view(-1, d))
+            ps = tq.Params(d, b + 1, m, R, S)
+            mse.append({"mse_bits": b, **quality.score_quality(ps, Q, K, quality.mse_only_keys(ps, codes, norm))})
         print(json.dumps({"workload": wl, "name": "attention quality, synthetic Qwen2.5-3B-shaped decode: "
                           "36 layers x 2 KV heads, 16 query heads, T8192, d128 (means over 576 query rows)",
                           "quality": res, "proj_dim_sweep_3bit_gaussian": sweep,
+                          "mse_only_keys_gaussian": mse,
                           "pages_qwen_validation": {"note": "real activations, not comparable",
                                                     "cosine": {"4": 0.999, "3": 0.995, "2": 0.988},
                                                     "top1": {"4": 0.87, "3": 0.82, "2": 0.66}}}), flush=True)

@@ -36,6 +36,27 @@ def exact_attention(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: fl
     return s, out
 
 
+def score_quality(p, q: torch.Tensor, K: torch.Tensor, keys, scale: float = 0.0):
+    """score_cosine and top1 of the compressed keys alone (no values)."""
+    B, Hq, Nq, d = q.shape
+    Hkv, T = K.shape[1], K.shape[2]
+    scale = scale if scale > 0 else 1.0 / math.sqrt(d)
+    est, _, _ = tq.tq_scores(p, q, keys, Hkv, T)
+    Kf = K.float().repeat_interleave(Hq // Hkv, dim=1)
+    cos, top1 = distribution_metrics(est, torch.matmul(q.float(), Kf.transpose(-1, -2)), scale)
+    return {"score_cosine": cos.mean().item(), "top1": top1.mean().item()}
+
+
+def mse_only_keys(p_scorer, codes: torch.Tensor, norm: torch.Tensor):
+    """Keys compressed with b MSE bits and no QJL stage (tq_compress_values with b bits), as a key
+    cache for a scorer whose key codebook has the same b bits (parameters of b + 1 bits): a zero
+    residual norm removes the QJL term, leaving the MSE-only estimate ||k|| <R q, c[idx]>."""
+    n = norm.numel()
+    signs = torch.zeros((n, p_scorer.proj_dim // 32), dtype=torch.int32, device=codes.device)
+    rnorm = torch.zeros(n, dtype=torch.float16, device=codes.device)
+    return codes, signs, norm, rnorm
+
+
 def attention_quality(p, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, keys, values, scale: float = 0.0):
     """Quality of the compressed cache (keys, values: the outputs of tq_compress_keys /
     tq_compress_values of K and V viewed as [B * Hkv * T, d]) for the queries q.  Returns a dict

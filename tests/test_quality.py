@@ -69,3 +69,25 @@ def test_quality_against_oracle():
         got[bits] = g
     assert got[2]["score_cosine"] < got[3]["score_cosine"] < got[4]["score_cosine"]
     assert got[2]["out_cosine"] < got[3]["out_cosine"] < got[4]["out_cosine"]
+
+
+@pytest.mark.gpu
+def test_mse_only_keys_scores_match_dequantized_dot():
+    """MSE-only keys scored through tq_scores (zero residual norm, key codebook of the same bits)
+    equal q . dequantize(key) from the oracle, and differ from the two-stage estimate."""
+    import torch
+    from kv_cache_vector_compress_b200 import quality, tq
+    d, m, T, Hq = 128, 64, 700, 3
+    R, S = synth.rotation(d, 721), synth.gaussian(m, d, 722)
+    K = synth.gaussian(T, d, 723).astype(np.float16)
+    Q = synth.gaussian(Hq, d, 724).reshape(1, Hq, 1, d)
+    for b in (2, 3):
+        v = oracle.compress(K, R, None, b, is_key=False)
+        ref = Q.reshape(Hq, d).astype(np.float64) @ oracle.dequantize(v["codes"], v["norm"], R, b).T
+        ps = tq.Params(d, b + 1, m, torch.from_numpy(R).cuda(), torch.from_numpy(S).cuda())
+        codes = torch.from_numpy(v["codes"].view(np.int32)).cuda()
+        norm = torch.from_numpy(v["norm"].view(np.float16)).cuda()
+        s, _, _ = tq.tq_scores(ps, torch.from_numpy(Q).cuda(), quality.mse_only_keys(ps, codes, norm), 1, T)
+        torch.cuda.synchronize()
+        from .parity import check_close
+        check_close(s[0, :, 0], ref, f"MSE-only scores, {b} bits")
