@@ -29,13 +29,9 @@ using namespace sm100;
 
 constexpr int kTileRows = 128;
 constexpr int kEpiWarp0 = 2;   // warps 2..9: epilogue (two groups of four)
-constexpr int kNormWarp0 = 10; // warps 10..: row norms of the input tiles
-// Row-norm warps: four, one per SM sub-partition, so the code step's sub-partitions carry equal
-// work; two for the register-heavy eight-level keys and sixteen-level values.
-template <bool IS_KEY, int BETA>
-constexpr int tc_norm_warps() { return (IS_KEY ? BETA == 3 : BETA == 4) ? 2 : 4; }
-template <bool IS_KEY, int BETA>
-constexpr int tc_threads() { return 32 * (kNormWarp0 + tc_norm_warps<IS_KEY, BETA>()); }
+constexpr int kEpiWarps = 8;   // warps 2..9
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+
 constexpr int kEScaleLog2 = 14;  // residual scale before the fp16 hi/lo split
 
 struct TcSmem {
@@ -54,7 +50,7 @@ __host__ __device__ inline int tc_rotation_slots(int D, int m, bool is_key) {
 }
 
 // misc block: codebook and flags (256 B), squared row norms [4][128], half residual norms [4][128]
-constexpr uint32_t kMiscNorm = 256, kMiscEe = 256 + 2048;
+constexpr uint32_t kMiscNorm = 256, kMiscEe = 256 + 4096;
 constexpr uint32_t kMiscBytes = kMiscEe + 2048;
 
 __host__ __device__ inline TcSmem tc_smem_layout(int D, int m, bool is_key) {
@@ -86,7 +82,7 @@ enum BarIdx {
     kEmpty = 5,      // [4] input stage consumed (rotation + both norm warps)
     kRotFull = 9,    // [4] rotation accumulator ready
     kEReady = 13,    // [4] codes written; keys: residual in TMEM; values: accumulator free
-    kNormReady = 17, // [4] squared row norms of the slot's tile
+    kNormReady = 17, // [4] both halves' squared row norms of the slot's tile
     kPartReady = 21, // [4] half-1 residual norms handed to half 0
     kProjFull = 25,  // [2] projection accumulator ready (and its residual operand consumed)
     kAccFree = 27    // [2] projection accumulator read
@@ -111,7 +107,7 @@ __device__ __forceinline__ void magnitude_bits(float u, const float *e, bool (&m
 }
 
 template <int D, bool IS_KEY, int BETA>
-__global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
+__global__ void __launch_bounds__(kThreads, 1)
     compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, Prepared P, int64_t n,
                        uint32_t *__restrict__ codes, uint32_t *__restrict__ signs, uint16_t *__restrict__ norm,
                        uint16_t *__restrict__ rnorm, int32_t *__restrict__ dev_status) {
@@ -121,7 +117,6 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
     const int m = IS_KEY ? P.m : 0;
     const TcSmem L = tc_smem_layout(D, m, IS_KEY);
     const int NST = L.nst, NRS = L.nrs;
-    constexpr int NW = tc_norm_warps<IS_KEY, BETA>();
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -130,7 +125,7 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
     float *cen_s = bnd_s + kMaxLevels;
     uint32_t *tmem_s = (uint32_t *)(cen_s + kMaxLevels);
     volatile int *abort_s = (volatile int *)(tmem_s + 1);
-    float *norm_s = (float *)(sm + L.misc + kMiscNorm);    // [slot][row] squared norms
+    float *norm_s = (float *)(sm + L.misc + kMiscNorm);    // [half][slot][row] partial squared norms
     float *ee_s = (float *)(sm + L.misc + kMiscEe);        // [slot][row] half residual norms
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -141,10 +136,10 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
         mbar_init(&bars[kOpnd], 1);
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars[kFull + s], 1);
-            mbar_init(&bars[kEmpty + s], 1 + NW);  // MMA commit + the norm warps
+            mbar_init(&bars[kEmpty + s], 1);  // MMA commit
             mbar_init(&bars[kRotFull + s], 1);
             mbar_init(&bars[kEReady + s], 8);
-            mbar_init(&bars[kNormReady + s], NW);
+            mbar_init(&bars[kNormReady + s], kEpiWarps);
             mbar_init(&bars[kPartReady + s], 4);
         }
         for (int s = 0; s < 2; ++s) {
@@ -267,7 +262,7 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
                 for (int i = 0; ok && i < my_tiles; ++i) ok = rotation(i);
             }
         }
-    } else if (warp < kNormWarp0) {
+    } else if (warp < kEpiWarp0 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue
         // Every tile goes to all eight warps: warp (q, h) takes rows 32q..32q+31 (its TMEM lane
         // quarter) and half h of the coordinates and of the projections.  Keys run the code step
@@ -299,10 +294,32 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
             const int64_t v = tile * kTileRows + row;
             const bool valid = v < n;
-            if (!mbar_wait(&bars[kNormReady + rs], ph, abort_s)) return false;
             if (!mbar_wait(&bars[kRotFull + rs], ph, abort_s)) return false;
             tc_fence_after();
-            const float nx = sqrtf(norm_s[rs * kTileRows + row]);
+            const uint32_t tl = tmem + lanes + rs * D;
+            // ||x|| = ||R x|| (R orthogonal, to the 2^-22 of its split) from the accumulator: each
+            // half of the row sums its squares, the halves meet in shared memory.  norm_s[.][rs] is
+            // next written NRS tiles on, after every warp has released this slot.
+            {
+                uint32_t r[32];
+                float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll 1
+                for (int c = h * CH; c < h * CH + CH; ++c) {
+                    tmem_ld32(tl + 32 * c, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float2 a2 = make_float2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+                        ss2 = __ffma2_rn(a2, a2, ss2);
+                    }
+                }
+                norm_s[(h * 4 + rs) * kTileRows + row] = ss2.x + ss2.y;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kNormReady + rs]);
+                if (!mbar_wait(&bars[kNormReady + rs], ph, abort_s)) return false;
+            }
+            const float nx = sqrtf(norm_s[rs * kTileRows + row] + norm_s[(4 + rs) * kTileRows + row]) *
+                             (1.0f / (float)(1 << kRScaleLog2));
             // the accumulator holds 2^8 R x; y = R x / ||x||
             const float inv = nx > 0.f ? (1.0f / (float)(1 << kRScaleLog2)) / nx : 0.f;
             const float inve = inv * (float)(1 << kEScaleLog2);
@@ -313,7 +330,6 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
 #pragma unroll
             for (int k = 0; k < HL - 1; ++k) ep[k] = edge[k] * sc;
             float2 ee2 = make_float2(0.f, 0.f);  // sums of (2^14 (y - c))^2 over even / odd coordinates
-            const uint32_t tl = tmem + lanes + rs * D;
             uint32_t *dst = codes + v * wpv;
             uint32_t r[32];
             // the loop stays rolled so the unrolled body fits the instruction cache
@@ -435,42 +451,6 @@ __global__ void __launch_bounds__(tc_threads<IS_KEY, BETA>(), 1)
             for (int i = 0; i < my_tiles; ++i)
                 if (!code_step(i)) break;
         }
-    } else {
-        // ------------------------------------------------------------ row norms
-        // ||x||^2 of every row of the fp16 input tile, read from the swizzled stage in
-        // shared memory (exact fp16 inputs, fp32 sums of even and odd coordinates); NW warps,
-        // 128 / NW rows each.  Slot rs of
-        // norm_s is rewritten once the code step of the tile NRS earlier has read it.
-        const int nw = warp - kNormWarp0;
-        for (int i = 0; i < my_tiles; ++i) {
-            const int rs = i % NRS, stage = i % NST;
-            if (i >= NRS && !mbar_wait(&bars[kEReady + rs], ((i / NRS) - 1) & 1, abort_s)) break;
-            if (!mbar_wait(&bars[kFull + stage], (i / NST) & 1, abort_s)) break;
-            const uint8_t *xs = sm + L.X + stage * XSTAGE;
-#pragma unroll
-            for (int hh = 0; hh < 4 / NW; ++hh) {
-                const int r = nw * (kTileRows / NW) + hh * 32 + lane;
-                float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    const int kb = c >> 3, cc = c & 7;
-                    const uint4 w = *(const uint4 *)(xs + kb * (kTileRows * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
-                    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __half22float2(*(const __half2 *)&u[e]);
-                        ss2 = __ffma2_rn(f, f, ss2);
-                    }
-                }
-                const float ss = ss2.x + ss2.y;
-                norm_s[rs * kTileRows + r] = ss;
-            }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars[kNormReady + rs]);
-                mbar_arrive(&bars[kEmpty + stage]);
-            }
-        }
     }
 
     tc_fence_before();
@@ -518,7 +498,7 @@ cudaError_t launch_tc(const Prepared &P, const void *x, int64_t n, uint32_t *cod
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    compress_tc_kernel<D, IS_KEY, BETA><<<grid, tc_threads<IS_KEY, BETA>(), smem, s>>>(map, P, n, codes, signs, norm, rnorm,
+    compress_tc_kernel<D, IS_KEY, BETA><<<grid, kThreads, smem, s>>>(map, P, n, codes, signs, norm, rnorm,
                                                                    dev_status);
     return cudaGetLastError();
 }
