@@ -44,14 +44,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-// The waiting thread is suspended (it issues nothing) until the phase completes or about 1 ms
-// has passed, so spinning warps do not take issue slots from the working ones.
+// (A suspend-time hint on this wait measured about 1% slower in the compress kernels.)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(addr), "r"(parity), "r"(1000000u)
+        : "r"(addr), "r"(parity)
         : "memory");
     return ok != 0;
 }
