@@ -356,10 +356,14 @@ def run_workload(args):
     per-op device time with CUDA events after warm-up, rates, and HBM fractions."""
     import numpy as np
     import torch
+    from kv_cache_vector_compress_b200 import dist as tqdist
     from kv_cache_vector_compress_b200 import synth, tq
-    torch.cuda.set_device(0)
+    ri = tqdist.rank_info()
+    torch.cuda.set_device(ri.local)
     pk = peaks()
     wl = args.workload
+    if ri.world > 1 and wl != 5:
+        raise SystemExit("only the vector-search workload (5) shards over ranks; the others run on one GPU")
     s = synth.seeds(wl)
     st = torch.cuda.current_stream()
 
@@ -447,31 +451,55 @@ def run_workload(args):
     elif wl == 5:
         d, m, bits, Nq, k = 1024, 512, 4, 1024, 10
         N = args.db if args.db > 0 else 1_000_000
+        # with several ranks the database of N keys is sharded (contiguous rows per rank, each
+        # shard generated from its own seed); the per-rank top-k lists meet in sharded_topk
+        tqdist.init("nccl", timeout_s=120)
+        start, Nl = tqdist.shard(N, ri.world, ri.rank)
         R = torch.from_numpy(synth.rotation(d, s["R"])).cuda()
         S = torch.from_numpy(synth.gaussian(m, d, s["S"])).cuda()
         p = tq.Params(d, bits, m, R, S)
-        X = synth.torch_normal_f32((N, d), s["keys"])
+        X = synth.torch_normal_f32((Nl, d), s["keys"] + tqdist.seed_offset(ri.rank))
         X /= X.norm(dim=1, keepdim=True)
         Qv = synth.torch_normal_f32((1, 1, Nq, d), s["queries"])
         Qv /= Qv.norm(dim=-1, keepdim=True)
         keys = tq.tq_compress_keys(p, X)
         kb = (bits - 1) * d // 8 + m // 8 + 4
-        ms = timed(lambda: tq.tq_compress_keys(p, X, *keys), steps=2, warmup=1)
+
+        def timed_ranks(fn, steps, warmup):
+            # device time on every rank between barriers; the slowest rank's time is reported
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize()
+            tqdist.barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            for _ in range(steps):
+                fn()
+            b.record(st)
+            torch.cuda.synchronize()
+            tqdist.barrier()
+            return tqdist.max_over_ranks(a.elapsed_time(b) / steps, device="cuda")
+        ms = timed_ranks(lambda: tq.tq_compress_keys(p, X, *keys), steps=2, warmup=1)
         out.append(rec("compress_db", ms, N, "vectors", N * (4 * d + kb)))
         ti = torch.empty((1, 1, Nq, k), dtype=torch.int32, device="cuda")
         tv = torch.empty((1, 1, Nq, k), dtype=torch.float32, device="cuda")
-        scr = torch.empty(tq.tq_scores_scratch_bytes(p, 1, 1, 1, Nq, N, k), dtype=torch.uint8, device="cuda")
-        ms = timed(lambda: tq.tq_scores(p, Qv, keys, 1, N, want_scores=False, topk=k, topk_idx=ti, topk_val=tv,
-                                        scratch=scr), steps=5, warmup=3)
+        scr = torch.empty(tq.tq_scores_scratch_bytes(p, 1, 1, 1, Nq, Nl, k), dtype=torch.uint8, device="cuda")
+
+        def search():
+            tq.tq_scores(p, Qv, keys, 1, Nl, want_scores=False, topk=k, topk_idx=ti, topk_val=tv, scratch=scr)
+            if ri.world > 1:
+                tqdist.sharded_topk(ti.view(Nq, k), tv.view(Nq, k), k, start)
+        ms = timed_ranks(search, steps=5, warmup=3)
         r = rec("scores_top10", ms, N * Nq, "query_key_pairs", N * kb)
         r["tflops_equiv"] = 2.0 * Nq * N * (d + m) / (ms * 1e-3) / 1e12
         # tensor-core work actually issued: fp16 hi/lo split products, 3 per centroid column and
         # 2 per sign column, on 128-padded tiles
         pad = lambda x: (x + 127) // 128 * 128
         r["tflops_mma"] = 2.0 * pad(Nq) * pad(N) * (3 * d + 2 * m) / (ms * 1e-3) / 1e12
-        r["frac_tensor"] = r["tflops_mma"] / pk["bf16_tflops"] if pk.get("bf16_tflops") else None
+        r["frac_tensor"] = r["tflops_mma"] / (ri.world * pk["bf16_tflops"]) if pk.get("bf16_tflops") else None
         out.append(r)
-        name = f"vector search: {N} x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
+        name = (f"vector search: {N} x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
+                + (f", sharded over {ri.world} GPUs (per-rank top-k lists gathered and merged)" if ri.world > 1 else ""))
     elif wl == 6:
         # one decode step on the decode-attention shape: append the new token of every (batch, KV
         # head) into slot t of a cache of capacity T, then attend over slots 0..t
@@ -556,7 +584,10 @@ def run_workload(args):
         return 0
     else:
         raise SystemExit("unknown workload")
-    print(json.dumps({"workload": wl, "name": name, "ops": out, "peak_hbm_gbs": pk["hbm_gbs"]}), flush=True)
+    if ri.rank == 0:
+        print(json.dumps({"workload": wl, "name": name, "ops": out, "n_gpus": ri.world,
+                          "peak_hbm_gbs": pk["hbm_gbs"]}), flush=True)
+    tqdist.destroy()
     return 0
 
 

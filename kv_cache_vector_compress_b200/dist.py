@@ -1,8 +1,10 @@
 """Host-side multi-GPU plumbing: one process per GPU, independent work per rank.
 
 The compression path partitions into independent (batch, KV-head) slices, so ranks share no data
-and no collective runs on the data path.  The only collective is the timing reduction: the
-reported time of a timed region is the maximum over ranks.
+and no collective runs on the data path; the timing reduction (the reported time of a timed
+region is the maximum over ranks) is the only collective there.  Vector search over a database
+sharded across ranks has one real exchange: every rank's top-k list of each query is gathered and
+merged (sharded_topk).
 """
 from __future__ import annotations
 
@@ -64,6 +66,31 @@ def shard(n: int, world: int, rank: int) -> tuple[int, int]:
 def weak_scaling_value(units_per_rank: int, world: int, max_seconds: float) -> float:
     """Whole-job throughput: all ranks' units over the slowest rank's time."""
     return world * units_per_rank / max_seconds
+
+
+def merge_topk(vals: torch.Tensor, idx: torch.Tensor, k: int):
+    """The k best of candidate lists [..., n] (score, key index) in the order of the top-k step:
+    score descending, ties to the smaller index.  Returns (idx, vals) [..., k]."""
+    o = torch.argsort(idx, dim=-1, stable=True)
+    v1, i1 = vals.gather(-1, o), idx.gather(-1, o)
+    o2 = torch.argsort(v1, dim=-1, descending=True, stable=True)
+    return i1.gather(-1, o2)[..., :k], v1.gather(-1, o2)[..., :k]
+
+
+def sharded_topk(local_idx: torch.Tensor, local_val: torch.Tensor, k: int, offset: int):
+    """Global top-k of a database sharded over the ranks.  Each rank passes the top-k of its own
+    shard (indices local to the shard, which starts at key `offset`); the lists are gathered from
+    all ranks (one all_gather each for indices and scores) and merged.  Every rank returns the
+    global (idx, vals) [..., k]."""
+    gidx = local_idx.to(torch.int64) + offset
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return merge_topk(local_val, gidx, k)
+    world = dist.get_world_size()
+    all_v = [torch.empty_like(local_val) for _ in range(world)]
+    all_i = [torch.empty_like(gidx) for _ in range(world)]
+    dist.all_gather(all_v, local_val.contiguous())
+    dist.all_gather(all_i, gidx.contiguous())
+    return merge_topk(torch.cat(all_v, dim=-1), torch.cat(all_i, dim=-1), k)
 
 
 def destroy():

@@ -77,3 +77,42 @@ def test_shards_cover_every_unit_once(n, world):
 def test_single_rank_is_identity():
     assert tqdist.max_over_ranks(3.5) == 3.5
     assert tqdist.rank_info().world >= 1
+
+
+def _topk_worker(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import torch
+    tqdist.init("gloo", timeout_s=60)
+    nq, n, k = 5, 1003, 10
+    g = np.random.Generator(np.random.PCG64(77))
+    full = np.round(g.standard_normal((nq, n)), 1).astype(np.float32)  # many exact ties
+    start, cnt = tqdist.shard(n, world, rank)
+    local = torch.from_numpy(full[:, start:start + cnt])
+    # the shard's own top-k, as the search kernel returns it (local indices)
+    li, lv = tqdist.merge_topk(local, torch.arange(cnt, dtype=torch.int64).expand(nq, cnt), k)
+    gi, gv = tqdist.sharded_topk(li, lv, k, start)
+    out_q.put((rank, gi.numpy(), gv.numpy(), full))
+    tqdist.destroy()
+
+
+def test_sharded_topk_over_two_gloo_ranks():
+    """A database split over two ranks: the merged per-rank top-k lists equal the top-k of the whole
+    database (score descending, ties to the smaller index), on every rank."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_topk_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    full = res[0][3]
+    k = 10
+    for r in range(full.shape[0]):
+        order = np.lexsort((np.arange(full.shape[1]), -full[r]))[:k]
+        for _, gi, gv, _ in res:
+            assert np.array_equal(gi[r], order), (r, gi[r], order)
+            assert np.array_equal(gv[r], full[r, order])
