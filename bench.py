@@ -379,10 +379,12 @@ def run_workload(args):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / steps
 
-    def rec(op, ms, units, unit, nbytes):
+    def rec(op, ms, units, unit, nbytes, gpus=1):
+        # nbytes and units are whole-job figures; the HBM fraction is taken against the peak of
+        # all `gpus` devices that shared the work
         gbs = nbytes / (ms * 1e-3) / 1e9
         return {"op": op, "ms": ms, "units": units, f"{unit}_per_s": units / (ms * 1e-3), "GB/s": gbs,
-                "frac_hbm": gbs / pk["hbm_gbs"]}
+                "frac_hbm": gbs / (gpus * pk["hbm_gbs"])}
 
     out = []
     if wl == 1:
@@ -480,7 +482,7 @@ def run_workload(args):
             tqdist.barrier()
             return tqdist.max_over_ranks(a.elapsed_time(b) / steps, device="cuda")
         ms = timed_ranks(lambda: tq.tq_compress_keys(p, X, *keys), steps=2, warmup=1)
-        out.append(rec("compress_db", ms, N, "vectors", N * (4 * d + kb)))
+        out.append(rec("compress_db", ms, N, "vectors", N * (4 * d + kb), gpus=ri.world))
         ti = torch.empty((1, 1, Nq, k), dtype=torch.int32, device="cuda")
         tv = torch.empty((1, 1, Nq, k), dtype=torch.float32, device="cuda")
         scr = torch.empty(tq.tq_scores_scratch_bytes(p, 1, 1, 1, Nq, Nl, k), dtype=torch.uint8, device="cuda")
@@ -490,7 +492,7 @@ def run_workload(args):
             if ri.world > 1:
                 tqdist.sharded_topk(ti.view(Nq, k), tv.view(Nq, k), k, start)
         ms = timed_ranks(search, steps=5, warmup=3)
-        r = rec("scores_top10", ms, N * Nq, "query_key_pairs", N * kb)
+        r = rec("scores_top10", ms, N * Nq, "query_key_pairs", N * kb, gpus=ri.world)
         r["tflops_equiv"] = 2.0 * Nq * N * (d + m) / (ms * 1e-3) / 1e12
         # tensor-core work actually issued: fp16 hi/lo split products, 3 per centroid column and
         # 2 per sign column, on 128-padded tiles

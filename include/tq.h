@@ -235,7 +235,10 @@ tq_status tq_selftest_wait_timeout(int32_t *dev_status, uint32_t timeout_ms, tq_
  *     with TQ_ERR_UNSUPPORTED before any work; use tq_attend with your own scratch for them.
  *   - The call never allocates: no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's address on that device (with that device
- *     current); make that first call before any stream capture.
+ *     current); make that first call before any stream capture.  The address is kept for the
+ *     life of the process and belongs to the device's primary context (the one the CUDA runtime
+ *     uses): do not call this after cudaDeviceReset, or with a different driver context current
+ *     on that device.
  *   - All calls share the one array, which keeps the last call's contents (nothing in it needs
  *     to start at zero).  Calls whose work overlaps on the GPU (other streams, other host
  *     threads) race on it: serialise them.
