@@ -168,6 +168,7 @@ size_t tq_scores_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int N
     const ScoresPlan plan = plan_scores(P, sp, topk);
     size_t bytes = qprep_bytes(P, sp);
     if (plan.search) bytes += search_scratch_bytes(P, sp, plan.fused_topk ? topk : 0);
+    if (plan.planes) bytes += planes_frag_bytes(P, sp);
     if (topk > 0 && !plan.fused_topk) bytes += topk_scratch_bytes(P, sp, topk);
     return bytes;
 }
@@ -196,9 +197,11 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     cur += qprep_bytes(P, sp);
     void *search_scratch = cur;
     if (plan.search) cur += search_scratch_bytes(P, sp, plan.fused_topk ? topk : 0);
+    uint32_t *frag = (uint32_t *)cur;
+    if (plan.planes) cur += planes_frag_bytes(P, sp);
     float *sbuf = scores;
     if (!sbuf && !plan.fused_topk) sbuf = (float *)cur;
-    cudaError_t e = launch_qprep(P, sp, qprep, s);
+    cudaError_t e = plan.planes ? cudaSuccess : launch_qprep(P, sp, qprep, s);
     if (e != cudaSuccess) return from_cuda(e);
     if (plan.fused_topk) {
         e = launch_search(P, sp, qprep, search_scratch, scores, topk, topk_idx, topk_val, dev_status, s);
@@ -206,6 +209,8 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     }
     if (plan.search)
         e = launch_search(P, sp, qprep, search_scratch, sbuf, 0, nullptr, nullptr, dev_status, s);
+    else if (plan.planes)
+        e = launch_planes(P, sp, 1.0f, frag, plan_planes(sp), false, sbuf, nullptr, s);
     else if (plan.mma)
         e = launch_decode_mma(P, sp, qprep, 1.0f, sbuf, decode_mma_splits(sp), false, s);
     else
@@ -221,7 +226,8 @@ size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int N
     ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                    nullptr);
     const AttendPlan plan = plan_attend(P, sp);
-    return qprep_bytes(P, sp) + attend_partials_bytes(P, sp, plan.splits);
+    return qprep_bytes(P, sp) + attend_partials_bytes(P, sp, plan.splits) +
+           (plan.planes ? planes_frag_bytes(P, sp) : 0);
 }
 
 tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
@@ -246,9 +252,12 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     float *qprep = (float *)scratch;
     const AttendPlan plan = plan_attend(P, sp);
     float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
-    cudaError_t e = launch_qprep(P, sp, qprep, s);
+    uint32_t *frag = (uint32_t *)((char *)partials + attend_partials_bytes(P, sp, plan.splits));
+    cudaError_t e = plan.planes ? cudaSuccess : launch_qprep(P, sp, qprep, s);
     if (e == cudaSuccess) {
-        if (plan.mma) {
+        if (plan.planes) {
+            e = launch_planes(P, sp, scale, frag, plan.pp, true, out, partials, s);
+        } else if (plan.mma) {
             e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
             if (e == cudaSuccess) e = launch_attend_combine(P, sp, partials, plan.splits, out, s);
         } else {
@@ -295,8 +304,15 @@ tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new
     cudaStream_t s = (cudaStream_t)stream;
     float *qprep = (float *)scratch;
     float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
-    cudaError_t e = launch_qprep(P, sp, qprep, s);
-    if (plan.mma) {
+    uint32_t *frag = (uint32_t *)((char *)partials + attend_partials_bytes(P, sp, plan.splits));
+    cudaError_t e = plan.planes ? cudaSuccess : launch_qprep(P, sp, qprep, s);
+    if (plan.planes) {
+        // the append kernel, then the bit-plane attention over slots 0..t of the strided cache
+        if (e == cudaSuccess) e = launch_append(P, sp, s);
+        ScoreProblem rd = sp;
+        rd.knew = rd.vnew = nullptr;
+        if (e == cudaSuccess) e = launch_planes(P, rd, scale, frag, plan.pp, true, out, partials, s);
+    } else if (plan.mma) {
         // the append runs inside the attention kernel
         if (e == cudaSuccess) e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
         if (e == cudaSuccess) e = launch_attend_combine(P, sp, partials, plan.splits, out, s);

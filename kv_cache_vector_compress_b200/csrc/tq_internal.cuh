@@ -168,15 +168,34 @@ int decode_mma_splits(const ScoreProblem &sp);
 cudaError_t launch_decode_mma(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale,
                               float *out, int splits, bool attend, cudaStream_t s);
 
+// Bit-plane integer tensor-core attention and scores (tq_attend_planes.cu): up to four query
+// rows per KV head, head_dim 64/128/256 with proj_dim = head_dim / 2.
+struct PlanesPlan {
+    int range;   // tokens per CTA
+    int splits;  // CTAs per (batch, KV head)
+};
+bool planes_supported(const Prepared &P, const ScoreProblem &sp, bool attend);
+PlanesPlan plan_planes(const ScoreProblem &sp);
+size_t planes_frag_bytes(const Prepared &P, const ScoreProblem &sp);
+// Query operands (rotation and projection of the queries included), then scores (attend =
+// false: out = scores [B, Hq, Nq, T]) or the attention output (attend = true: out = [B, Hq, Nq, d],
+// through per-range partials [rows, splits, d + 2] that the last CTA of each slice merges).
+cudaError_t launch_planes(const Prepared &P, const ScoreProblem &sp, float scale, uint32_t *frag,
+                          const PlanesPlan &pl, bool attend, float *out, float *partials, cudaStream_t s);
+
 // Which attention kernel a problem uses and how many context splits it takes.
 struct AttendPlan {
+    bool planes;
     bool mma;
     int splits;
+    PlanesPlan pp;
 };
 inline AttendPlan plan_attend(const Prepared &P, const ScoreProblem &sp) {
     AttendPlan a;
-    a.mma = decode_mma_supported(P, sp, true);
-    a.splits = a.mma ? decode_mma_splits(sp) : attend_splits(sp);
+    a.planes = planes_supported(P, sp, true);
+    a.mma = !a.planes && decode_mma_supported(P, sp, true);
+    a.pp = plan_planes(sp);
+    a.splits = a.planes ? a.pp.splits : a.mma ? decode_mma_splits(sp) : attend_splits(sp);
     return a;
 }
 size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
@@ -193,13 +212,15 @@ cudaError_t launch_search(const Prepared &P, const ScoreProblem &sp, const float
 struct ScoresPlan {
     bool search;      // launch_search
     bool fused_topk;  // the search keeps the top-k itself
+    bool planes;      // launch_planes in scores mode
     bool mma;         // launch_decode_mma in scores mode
 };
 inline ScoresPlan plan_scores(const Prepared &P, const ScoreProblem &sp, int topk) {
     ScoresPlan a;
     a.fused_topk = topk > 0 && search_tc_supported(P, sp, topk);
     a.search = a.fused_topk || search_tc_supported(P, sp, 0);
-    a.mma = !a.search && decode_mma_supported(P, sp, false);
+    a.planes = !a.search && planes_supported(P, sp, false);
+    a.mma = !a.search && !a.planes && decode_mma_supported(P, sp, false);
     return a;
 }
 

@@ -383,29 +383,59 @@ __global__ void __launch_bounds__(kTile) attend_kernel(Prepared P, ScoreProblem 
     (void)rows_total;
 }
 
-__global__ void attend_combine_kernel(Prepared P, int64_t rows, int splits,
-                                      const float *__restrict__ partials, float *__restrict__ out) {
-    extern __shared__ float orot[];
+// Merge the split-context partials (max, sum, o_rot) of each query row and rotate back:
+// out = R^T (sum_s e^{M_s - M} o_s) / (sum_s e^{M_s - M} l_s).  One block per row; the split loads
+// of a coordinate are issued eight at a time.
+__global__ void __launch_bounds__(128) attend_combine_kernel(Prepared P, int64_t rows, int splits,
+                                                             const float *__restrict__ partials,
+                                                             float *__restrict__ out) {
+    extern __shared__ float csm[];
     const int d = P.d;
+    float *orot = csm;     // [d]
+    float *wts = csm + d;  // [splits]
+    __shared__ float lsum;
     for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
         const float *pp = partials + row * splits * (int64_t)(d + 2);
-        float M = -INFINITY;
-        for (int s = 0; s < splits; ++s) M = fmaxf(M, pp[(int64_t)s * (d + 2)]);
-        for (int j = threadIdx.x; j < d; j += blockDim.x) {
-            float acc = 0.f, L = 0.f;
-            for (int s = 0; s < splits; ++s) {
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            float M = -INFINITY;
+            for (int s = lane; s < splits; s += 32) M = fmaxf(M, pp[(int64_t)s * (d + 2)]);
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            float L = 0.f;
+            for (int s = lane; s < splits; s += 32) {
                 const float *ps = pp + (int64_t)s * (d + 2);
                 const float w = (ps[0] == -INFINITY) ? 0.f : expf(ps[0] - M);
-                acc = fmaf(w, ps[2 + j], acc);
+                wts[s] = w;
                 L = fmaf(w, ps[1], L);
             }
-            orot[j] = acc / L;
+            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            if (lane == 0) lsum = L;
+        }
+        __syncthreads();
+        const float invL = 1.f / lsum;
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            const float *pj = pp + 2 + j;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            int s = 0;
+            for (; s + 8 <= splits; s += 8) {
+                float v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = pj[(int64_t)(s + u) * (d + 2)];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] = fmaf(wts[s + u], v[u], acc[u]);
+            }
+            for (; s < splits; ++s) acc[0] = fmaf(wts[s], pj[(int64_t)s * (d + 2)], acc[0]);
+            orot[j] = (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]))) * invL;
         }
         __syncthreads();
         for (int j = threadIdx.x; j < d; j += blockDim.x) {
-            float acc = 0.f;
-            for (int i = 0; i < d; ++i) acc = fmaf(P.R[(int64_t)i * d + j], orot[i], acc);
-            out[row * d + j] = acc;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int i = 0; i < d; i += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] = fmaf(P.R[(int64_t)(i + u) * d + j], orot[i + u], acc[u]);
+            }
+            out[row * d + j] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
         __syncthreads();
     }
@@ -490,8 +520,14 @@ cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float
 cudaError_t launch_attend_combine(const Prepared &P, const ScoreProblem &sp, const float *partials, int splits,
                                   float *out, cudaStream_t s) {
     const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
-    int blocks = (int)(rows < 148 * 8 ? rows : 148 * 8);
-    attend_combine_kernel<<<blocks, 128, sizeof(float) * P.d, s>>>(P, rows, splits, partials, out);
+    const int blocks = (int)(rows < 148 * 16 ? rows : 148 * 16);
+    const size_t smem = sizeof(float) * ((size_t)P.d + (size_t)splits);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    attend_combine_kernel<<<blocks, 128, smem, s>>>(P, rows, splits, partials, out);
     return cudaGetLastError();
 }
 
