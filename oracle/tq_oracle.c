@@ -323,11 +323,15 @@ static void dequant_one(int dim, int beta, const float *R, const float *cc32, co
                         double scale, int *idx, double *out)
 {
     unpack_codes(words, dim, beta, idx);
-    for (int j = 0; j < dim; ++j) {
-        double acc = 0.0;
-        for (int i = 0; i < dim; ++i) acc += (double)R[(size_t)i * dim + j] * (double)cc32[idx[i]];
-        out[j] = scale * acc;
+    /* out[j] = scale * sum_i R[i][j] c[idx_i], summed over i in ascending order (rows of R are
+       walked in memory order; every out[j] sees the same sequence of additions as a column walk) */
+    for (int j = 0; j < dim; ++j) out[j] = 0.0;
+    for (int i = 0; i < dim; ++i) {
+        const double ci = (double)cc32[idx[i]];
+        const float *Ri = R + (size_t)i * dim;
+        for (int j = 0; j < dim; ++j) out[j] += (double)Ri[j] * ci;
     }
+    for (int j = 0; j < dim; ++j) out[j] *= scale;
 }
 
 /* Dequantize n packed vectors to the original space (TurboQuantMSE.dequantize). */
