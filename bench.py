@@ -272,6 +272,20 @@ def run_tq(args):
         t1.record(stream)
         barrier()
     ms = t0.elapsed_time(t1)
+    # scores alone over the same cache (not part of the step): tq_scores into a [B, Hq, Nq, T] buffer
+    sc_buf = torch.empty((B, Hq, Nq, T), dtype=torch.float32, device="cuda")
+    sc_scr = torch.empty(tq.tq_scores_scratch_bytes(p, B, Hq, Hkv, Nq, T, 0), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        tq.tq_scores(p, Q, keys, Hkv, T, scores=sc_buf, scratch=sc_scr)
+    barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        tq.tq_scores(p, Q, keys, Hkv, T, scores=sc_buf, scratch=sc_scr)
+    s1.record(stream)
+    barrier()
+    scores_ms = s0.elapsed_time(s1) / args.steps
+    del sc_buf, sc_scr
     op_ms = {"compress_keys": 0.0, "compress_values": 0.0, "attend": 0.0}
     for e in evs:
         op_ms["compress_keys"] += e[0].elapsed_time(e[1]) / args.steps
@@ -323,6 +337,14 @@ def run_tq(args):
         breakdown["compress_keys"]["vectors_per_s"] = n / (op_ms["compress_keys"] * 1e-3)
         breakdown["compress_values"]["vectors_per_s"] = n / (op_ms["compress_values"] * 1e-3)
         breakdown["attend"]["packed_keys_scored_per_s"] = n / (op_ms["attend"] * 1e-3)
+        # scores only (outside the step): packed keys read, fp32 scores written
+        kbytes = n * record_bytes(w)[0]
+        sbytes = B * Hq * Nq * T * 4
+        sgbs = (kbytes + sbytes) / (scores_ms * 1e-3) / 1e9
+        breakdown["scores_only"] = {"ms": scores_ms, "algorithmic_bytes": kbytes + sbytes,
+                                    "bytes_note": "packed keys read + fp32 scores written", "GB/s": sgbs,
+                                    "frac_hbm": sgbs / pk["hbm_gbs"],
+                                    "packed_keys_scored_per_s": n / (scores_ms * 1e-3)}
         dom = max(op_ms, key=lambda k: op_ms[k])
         ach = ab[dom] / (op_ms[dom] * 1e-3) / 1e9
         tpu = traffic_per_unit(dom)
@@ -340,7 +362,8 @@ def run_tq(args):
             "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "keys/s",
                     "h2d_bytes_per_step": int(hK.numel() * 2 + hV.numel() * 2 + hQ.numel() * 4),
                     "d2h_bytes_per_step": int(hO.numel() * 4)},
-            "gpu_launches": 5 * args.steps,
+            # per step: compress keys, compress values, query operands + bit-plane attention
+            "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),
         }
         if cpu:

@@ -82,6 +82,18 @@ int tq_version(void);
 tq_status tq_codebook(int dim, int bits, float *boundaries, float *centroids);
 
 /*
+ * The same Lloyd-Max conditions under the exact law of one coordinate of a uniformly random
+ * unit vector in R^dim, density proportional to (1 - y^2)^((dim-3)/2) on (-1, 1): the
+ * "concentrated Beta" law of "TurboQuant er nå tilgjengelig som Python-bibliotek"
+ * (jansverre.net), section "Hva er TurboQuant, kort fortalt?".  N(0, 1/dim) is its large-dim
+ * limit.  HOST function, no device work.  Arguments as tq_codebook; dim >= 3.
+ */
+tq_status tq_codebook_beta(int dim, int bits, float *boundaries, float *centroids);
+
+/* Coordinate laws a parameter set's codebooks can be built for (tq_prepare_law). */
+enum { TQ_LAW_GAUSSIAN = 0, TQ_LAW_BETA = 1 };
+
+/*
  * Quantizer parameters.  R and S are caller-generated (the pages use a fixed random
  * orthogonal R and an i.i.d. N(0,1) matrix S; the library takes them as inputs).
  *   dim      : head dimension d; a multiple of 32, 32..1024
@@ -113,6 +125,13 @@ size_t tq_workspace_bytes(int dim, int bits, int proj_dim);
  * once per (R, S), and again whenever they change.  Enqueued on `stream`.
  */
 tq_status tq_prepare(const tq_params *p, int32_t *dev_status, tq_stream_t stream);
+
+/*
+ * tq_prepare with the codebooks of a chosen coordinate law: TQ_LAW_GAUSSIAN (what tq_prepare
+ * uses, tq_codebook) or TQ_LAW_BETA (tq_codebook_beta).  Every other call then quantizes,
+ * scores and dequantizes with those codebooks.  TQ_ERR_INVALID_ARG for any other law.
+ */
+tq_status tq_prepare_law(const tq_params *p, int law, int32_t *dev_status, tq_stream_t stream);
 
 /*
  * Compress n key vectors (TurboQuantProd.compress / TurboQuantCompressorV2;

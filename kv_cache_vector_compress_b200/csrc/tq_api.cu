@@ -91,6 +91,16 @@ tq_status tq_codebook(int dim, int bits, float *boundaries, float *centroids) {
     return TQ_OK;
 }
 
+tq_status tq_codebook_beta(int dim, int bits, float *boundaries, float *centroids) {
+    if (dim < 3 || bits < 1 || bits > 4 || !boundaries || !centroids) return TQ_ERR_INVALID_ARG;
+    double b[kMaxLevels], c[kMaxLevels];
+    if (lloyd_max_beta(dim, bits, b, c) < 0) return TQ_ERR_INVALID_ARG;
+    const int K = 1 << bits;
+    for (int k = 0; k < K - 1; ++k) boundaries[k] = (float)b[k];
+    for (int k = 0; k < K; ++k) centroids[k] = (float)c[k];
+    return TQ_OK;
+}
+
 size_t tq_workspace_bytes(int dim, int bits, int proj_dim) {
     if (dim < 32 || dim > kMaxDim || dim % 32 || bits < 1 || bits > 4) return 0;
     if (proj_dim < 0 || proj_dim > kMaxProj || proj_dim % 32) return 0;
@@ -98,16 +108,22 @@ size_t tq_workspace_bytes(int dim, int bits, int proj_dim) {
 }
 
 tq_status tq_prepare(const tq_params *p, int32_t *dev_status, tq_stream_t stream) {
+    return tq_prepare_law(p, TQ_LAW_GAUSSIAN, dev_status, stream);
+}
+
+tq_status tq_prepare_law(const tq_params *p, int law, int32_t *dev_status, tq_stream_t stream) {
     (void)dev_status;
     tq_status st = check_params(p, false);
     if (st != TQ_OK) return st;
+    if (law != TQ_LAW_GAUSSIAN && law != TQ_LAW_BETA) return TQ_ERR_INVALID_ARG;
     if (!p->R || !aligned16(p->R)) return TQ_ERR_INVALID_ARG;
     if (p->proj_dim > 0 && (!p->S || !aligned16(p->S))) return TQ_ERR_INVALID_ARG;
+    auto solve = law == TQ_LAW_BETA ? lloyd_max_beta : lloyd_max_gaussian;
     Codebooks cb;
     memset(&cb, 0, sizeof(cb));
     double b[kMaxLevels], c[kMaxLevels];
     const int K = 1 << p->bits;
-    if (lloyd_max_gaussian(p->dim, p->bits, b, c) < 0) return TQ_ERR_INVALID_ARG;
+    if (solve(p->dim, p->bits, b, c) < 0) return TQ_ERR_INVALID_ARG;
     for (int k = 0; k < K; ++k) {
         cb.vc[k] = (float)c[k];
         if (k < K - 1) cb.vb[k] = (float)b[k];
@@ -116,7 +132,7 @@ tq_status tq_prepare(const tq_params *p, int32_t *dev_status, tq_stream_t stream
     for (int k = K - 1; k < kMaxLevels; ++k) cb.vb[k] = INFINITY;
     if (p->bits >= 2) {
         const int Kk = K / 2;
-        if (lloyd_max_gaussian(p->dim, p->bits - 1, b, c) < 0) return TQ_ERR_INVALID_ARG;
+        if (solve(p->dim, p->bits - 1, b, c) < 0) return TQ_ERR_INVALID_ARG;
         for (int k = 0; k < Kk; ++k) {
             cb.kc[k] = (float)c[k];
             if (k < Kk - 1) cb.kb[k] = (float)b[k];

@@ -122,6 +122,7 @@ inline Prepared prepared_view(const tq_params *p) {
 
 // Host-side Lloyd-Max (tq_codebook.cpp).
 int lloyd_max_gaussian(int dim, int bits, double *bounds, double *cents);
+int lloyd_max_beta(int dim, int bits, double *bounds, double *cents);
 
 // Kernel launchers (tq_*.cu).  All return a cudaError_t from cudaGetLastError.
 cudaError_t launch_prepare(const tq_params *p, const Codebooks &cb, cudaStream_t s);

@@ -113,3 +113,16 @@ def torch_normal_f32(shape, seed: int, device="cuda"):
     g = torch.Generator(device=device)
     g.manual_seed(seed)
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+
+def random_packed_keys(n: int, d: int, beta: int, m: int, seed: int, rho=(0.17, 0.20)):
+    """Seeded packed key records without a compression step: uniformly random code and sign
+    words, key norms 1 (fp16 1.0, unit keys) and residual norms uniform in `rho` (fp16), in the
+    layout of the library's key arrays.  Used to check scoring and top-k at full size where
+    compressing the inputs on the host would take too long."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    codes = rng.integers(0, 1 << 32, size=(n, beta * d // 32), dtype=np.uint64).astype(np.uint32)
+    signs = rng.integers(0, 1 << 32, size=(n, m // 32), dtype=np.uint64).astype(np.uint32)
+    norm = np.full(n, 0x3C00, np.uint16)
+    rnorm = rng.uniform(rho[0], rho[1], size=n).astype(np.float16).view(np.uint16)
+    return {"codes": codes, "signs": signs, "norm": norm, "rnorm": rnorm}

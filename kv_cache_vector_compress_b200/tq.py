@@ -44,9 +44,13 @@ _lib.tq_status_string.restype = ctypes.c_char_p
 _lib.tq_version.restype = _I
 _lib.tq_codebook.argtypes = [_I, _I, _P, _P]
 _lib.tq_codebook.restype = _I
+_lib.tq_codebook_beta.argtypes = [_I, _I, _P, _P]
+_lib.tq_codebook_beta.restype = _I
 _lib.tq_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.tq_workspace_bytes.restype = _SZ
 _lib.tq_prepare.argtypes = [_PP, _P, _P]
+_lib.tq_prepare_law.argtypes = [_PP, _I, _P, _P]
+_lib.tq_prepare_law.restype = _I
 _lib.tq_prepare.restype = _I
 _lib.tq_compress_keys.argtypes = [_PP, _P, _I, _I64, _P, _P, _P, _P, _P, _P]
 _lib.tq_compress_keys.restype = _I
@@ -73,7 +77,11 @@ _lib.tq_selftest_wait_timeout.restype = _I
 
 TQ_STATIC_SCRATCH_BYTES = 16 << 20
 
-EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_workspace_bytes", "tq_prepare",
+TQ_LAW_GAUSSIAN, TQ_LAW_BETA = 0, 1
+LAWS = {"gaussian": TQ_LAW_GAUSSIAN, "beta": TQ_LAW_BETA}
+
+EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_codebook_beta", "tq_workspace_bytes",
+           "tq_prepare", "tq_prepare_law",
            "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores",
            "tq_attend_scratch_bytes", "tq_attend", "tq_append_attend", "tq_selftest_wait_timeout",
            "tq_attend_static"]
@@ -115,11 +123,20 @@ def tq_codebook(dim: int, bits: int):
     return b, c
 
 
+def tq_codebook_beta(dim: int, bits: int):
+    """Host Lloyd-Max codebook for the exact (Beta) coordinate law of a random unit vector in R^dim."""
+    K = 1 << bits
+    b = torch.zeros(K - 1, dtype=torch.float32)
+    c = torch.zeros(K, dtype=torch.float32)
+    _check(_lib.tq_codebook_beta(dim, bits, _ptr(b), _ptr(c)), "tq_codebook_beta")
+    return b, c
+
+
 class Params:
     """A prepared parameter set: owns the device workspace and keeps R and S alive."""
 
     def __init__(self, dim: int, bits: int, proj_dim: int, R: torch.Tensor, S: torch.Tensor | None,
-                 prepare: bool = True):
+                 prepare: bool = True, law: str = "gaussian"):
         dev = R.device
         self.R = R.to(torch.float32).contiguous()
         self.S = S.to(device=dev, dtype=torch.float32).contiguous() if S is not None else None
@@ -131,8 +148,9 @@ class Params:
                            self.S.data_ptr() if self.S is not None else None,
                            self.workspace.data_ptr(), nbytes)
         self.dim, self.bits, self.proj_dim = dim, bits, proj_dim
+        self.law = law
         if prepare:
-            tq_prepare(self)
+            tq_prepare(self, law=law)
 
     @property
     def ref(self):
@@ -145,8 +163,17 @@ class Params:
         return self.bits * self.dim // 32
 
 
-def tq_prepare(p: Params, dev_status: torch.Tensor | None = None):
-    _check(_lib.tq_prepare(p.ref, _ptr(dev_status), _stream()), "tq_prepare")
+def tq_prepare_law(p: Params, law: str, dev_status: torch.Tensor | None = None):
+    """Fill p's workspace with the codebooks of `law` ("gaussian" or "beta")."""
+    _check(_lib.tq_prepare_law(p.ref, LAWS[law], _ptr(dev_status), _stream()), "tq_prepare_law")
+
+
+def tq_prepare(p: Params, dev_status: torch.Tensor | None = None, law: str = "gaussian"):
+    """Fill p's workspace; law "gaussian" (tq_prepare) or "beta" (tq_prepare_law)."""
+    if law == "gaussian":
+        _check(_lib.tq_prepare(p.ref, _ptr(dev_status), _stream()), "tq_prepare")
+    else:
+        tq_prepare_law(p, law, dev_status)
 
 
 def _dtype_code(x: torch.Tensor) -> int:

@@ -51,15 +51,19 @@ def lib():
         L.ora_codebook.restype = I
         L.ora_codebook_f32.argtypes = [I, I, P, P]
         L.ora_codebook_f32.restype = I
+        L.ora_codebook_beta.argtypes = [I, I, P, P]
+        L.ora_codebook_beta.restype = I
+        L.ora_codebook_law_f32.argtypes = [I, I, I, P, P]
+        L.ora_codebook_law_f32.restype = I
         L.ora_pack_codes.argtypes = [P, I, I, P]
         L.ora_unpack_codes.argtypes = [P, I, I, P]
-        L.ora_compress.argtypes = [I, I, I, I, P, P, P, I, I64, P, P, P, P, P, P]
+        L.ora_compress.argtypes = [I, I, I, I, P, P, P, I, I64, P, P, P, P, P, P, I]
         L.ora_compress.restype = I
-        L.ora_dequantize.argtypes = [I, I, P, P, P, I64, P]
+        L.ora_dequantize.argtypes = [I, I, P, P, P, I64, P, I]
         L.ora_dequantize.restype = I
-        L.ora_scores.argtypes = [I, I, I, P, P, P, I, I, I, I, I64, P, P, P, P, P]
+        L.ora_scores.argtypes = [I, I, I, P, P, P, I, I, I, I, I64, P, P, P, P, P, I]
         L.ora_scores.restype = I
-        L.ora_attend.argtypes = [I, I, I, P, P, P, I, I, I, I, I64, P, P, P, P, P, P, D, P]
+        L.ora_attend.argtypes = [I, I, I, P, P, P, I, I, I, I, I64, P, P, P, P, P, P, D, P, I]
         L.ora_attend.restype = I
         L.ora_topk.argtypes = [P, I64, I64, I, P, P]
         L.ora_topk.restype = I
@@ -103,11 +107,26 @@ def codebook(dim: int, bits: int):
     return b, c, it
 
 
-def codebook_f32(dim: int, bits: int):
+def codebook_beta(dim: int, bits: int):
+    """Lloyd-Max codebook for the exact coordinate law of a random unit vector in R^dim (density
+    proportional to (1 - y^2)^((dim-3)/2)), in double: (boundaries[K-1], centroids[K], iterations)."""
+    K = 1 << bits
+    b = np.zeros(K - 1, np.float64)
+    c = np.zeros(K, np.float64)
+    it = lib().ora_codebook_beta(dim, bits, _p(b), _p(c))
+    if it < 0:
+        raise ValueError("codebook did not converge / bad arguments")
+    return b, c, it
+
+
+LAWS = {"gaussian": 0, "beta": 1}
+
+
+def codebook_f32(dim: int, bits: int, law: str = "gaussian"):
     K = 1 << bits
     b = np.zeros(K - 1, np.float32)
     c = np.zeros(K, np.float32)
-    if lib().ora_codebook_f32(dim, bits, _p(b), _p(c)) < 0:
+    if lib().ora_codebook_law_f32(dim, bits, LAWS[law], _p(b), _p(c)) < 0:
         raise ValueError("codebook did not converge / bad arguments")
     return b, c
 
@@ -127,7 +146,7 @@ def unpack_codes(words: np.ndarray, dim: int, beta: int) -> np.ndarray:
 
 
 def compress(x: np.ndarray, R: np.ndarray, S: np.ndarray | None, bits: int, is_key: bool,
-             want_y: bool = False, want_p: bool = False):
+             want_y: bool = False, want_p: bool = False, law: str = "gaussian"):
     """Compress rows of x ([n, dim], fp16 or fp32).  Returns a dict of packed arrays
     (codes, norm as fp16 bits; keys also signs and rnorm) plus optional y32 / p32."""
     x = np.ascontiguousarray(x)
@@ -155,7 +174,7 @@ def compress(x: np.ndarray, R: np.ndarray, S: np.ndarray | None, bits: int, is_k
     rc = lib().ora_compress(1 if is_key else 0, dim, bits, m, _p(R), _p(S) if is_key else None,
                             _p(xb), xf16, n, _p(codes), _p(signs), _p(norm), _p(rnorm),
                             _p(y32) if y32 is not None else None,
-                            _p(p32) if p32 is not None else None)
+                            _p(p32) if p32 is not None else None, LAWS[law])
     if rc:
         raise ValueError("ora_compress rejected its arguments")
     out = {"codes": codes, "norm": norm}
@@ -169,19 +188,19 @@ def compress(x: np.ndarray, R: np.ndarray, S: np.ndarray | None, bits: int, is_k
     return out
 
 
-def dequantize(codes: np.ndarray, norm: np.ndarray, R: np.ndarray, beta: int) -> np.ndarray:
+def dequantize(codes: np.ndarray, norm: np.ndarray, R: np.ndarray, beta: int, law: str = "gaussian") -> np.ndarray:
     codes = _c(codes, np.uint32)
     norm = _c(norm, np.uint16)
     R = _c(R, np.float32)
     n = norm.shape[0]
     dim = R.shape[0]
     out = np.zeros((n, dim), np.float64)
-    if lib().ora_dequantize(dim, beta, _p(R), _p(codes), _p(norm), n, _p(out)):
+    if lib().ora_dequantize(dim, beta, _p(R), _p(codes), _p(norm), n, _p(out), LAWS[law]):
         raise ValueError("bad arguments")
     return out
 
 
-def scores(q, R, S, bits, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm) -> np.ndarray:
+def scores(q, R, S, bits, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, law: str = "gaussian") -> np.ndarray:
     q = _c(q, np.float32)
     R = _c(R, np.float32)
     S = _c(S, np.float32)
@@ -190,14 +209,14 @@ def scores(q, R, S, bits, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm) -> n
     out = np.zeros((B, Hq, Nq, T), np.float64)
     rc = lib().ora_scores(dim, bits, m, _p(R), _p(S), _p(q), B, Hq, Hkv, Nq, T,
                           _p(_c(kcodes, np.uint32)), _p(_c(ksigns, np.uint32)),
-                          _p(_c(knorm, np.uint16)), _p(_c(krnorm, np.uint16)), _p(out))
+                          _p(_c(knorm, np.uint16)), _p(_c(krnorm, np.uint16)), _p(out), LAWS[law])
     if rc:
         raise ValueError("bad arguments")
     return out
 
 
 def attend(q, R, S, bits, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, vcodes, vnorm,
-           scale: float | None = None) -> np.ndarray:
+           scale: float | None = None, law: str = "gaussian") -> np.ndarray:
     q = _c(q, np.float32)
     R = _c(R, np.float32)
     S = _c(S, np.float32)
@@ -209,7 +228,8 @@ def attend(q, R, S, bits, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, vcod
     rc = lib().ora_attend(dim, bits, m, _p(R), _p(S), _p(q), B, Hq, Hkv, Nq, T,
                           _p(_c(kcodes, np.uint32)), _p(_c(ksigns, np.uint32)),
                           _p(_c(knorm, np.uint16)), _p(_c(krnorm, np.uint16)),
-                          _p(_c(vcodes, np.uint32)), _p(_c(vnorm, np.uint16)), float(scale), _p(out))
+                          _p(_c(vcodes, np.uint32)), _p(_c(vnorm, np.uint16)), float(scale), _p(out),
+                          LAWS[law])
     if rc:
         raise ValueError("bad arguments")
     return out

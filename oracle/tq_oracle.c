@@ -162,6 +162,133 @@ int ora_codebook(int dim, int bits, double *bounds, double *cents)
     return it;
 }
 
+/*
+ * Lloyd-Max quantizer for the exact law of one coordinate of a uniformly random unit vector
+ * in R^dim, which [P5] "Hva er TurboQuant, kort fortalt?" describes as a concentrated Beta law:
+ * y = 2 B - 1 with B ~ Beta((dim-1)/2, (dim-1)/2), i.e. density proportional to
+ * (1 - y^2)^((dim-3)/2) on (-1, 1).  (N(0, 1/dim) is its large-dim limit.)
+ *
+ * The same two conditions as above, alternated until nothing moves:
+ *   boundary_k = (c_k + c_{k+1}) / 2,   c_k = E[y | b_{k-1} < y < b_k]   (b_{-1} = -1, b_{K-1} = 1)
+ * The conditional mean is (int y f) / (int f) over the cell.  With y = sin(theta) both integrals
+ * become integrals of smooth functions of theta, int cos^(dim-2) and int sin cos^(dim-2), taken
+ * by composite 16-point Gauss-Legendre quadrature on panels no wider than 1/(2 sqrt(dim)).
+ * Returns the number of iterations, or -1 on bad arguments / no convergence.
+ */
+static double gl_x[16], gl_w[16];
+static int gl_ready = 0;
+
+static void gauss_legendre16(void)
+{
+    /* nodes: roots of P_16 by Newton's method; weights 2 / ((1 - x^2) P_16'(x)^2) */
+    const int n = 16;
+    for (int i = 0; i < n / 2; ++i) {
+        double z = cos(ORA_PI * (i + 0.75) / (n + 0.5)), dp = 0.0;
+        for (int it = 0; it < 100; ++it) {
+            double p0 = 1.0, p1 = z;
+            for (int k = 2; k <= n; ++k) {
+                const double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+                p0 = p1;
+                p1 = p2;
+            }
+            dp = n * (z * p1 - p0) / (z * z - 1.0);
+            const double dz = p1 / dp;
+            z -= dz;
+            if (fabs(dz) < 1e-16) break;
+        }
+        gl_x[i] = -z;
+        gl_x[n - 1 - i] = z;
+        gl_w[i] = gl_w[n - 1 - i] = 2.0 / ((1.0 - z * z) * dp * dp);
+    }
+    gl_ready = 1;
+}
+
+/* mass and first moment of the law over (lo, hi), up to the common normalising constant */
+static void beta_cell(int dim, double lo, double hi, double *mass, double *moment)
+{
+    const double t0 = asin(lo), t1 = asin(hi);
+    double hmax = 0.5 / sqrt((double)dim);
+    if (hmax > 0.05) hmax = 0.05;
+    int panels = (int)ceil((t1 - t0) / hmax);
+    if (panels < 1) panels = 1;
+    const double h = (t1 - t0) / panels;
+    double m0 = 0.0, m1 = 0.0;
+    for (int p = 0; p < panels; ++p) {
+        const double mid = t0 + (p + 0.5) * h;
+        for (int i = 0; i < 16; ++i) {
+            const double th = mid + 0.5 * h * gl_x[i];
+            const double w = 0.5 * h * gl_w[i] * pow(cos(th), dim - 2);
+            m0 += w;
+            m1 += w * sin(th);
+        }
+    }
+    *mass = m0;
+    *moment = m1;
+}
+
+int ora_codebook_beta(int dim, int bits, double *bounds, double *cents)
+{
+    if (dim < 2 || bits < 1 || bits > 8) return -1;
+    if (!gl_ready) gauss_legendre16();
+    const int K = 1 << bits;
+    double *c = (double *)malloc(sizeof(double) * K);
+    double *b = (double *)malloc(sizeof(double) * (K + 1));
+    double spread = 3.0 / sqrt((double)dim);
+    if (spread > 0.9) spread = 0.9;
+    for (int k = 0; k < K; ++k) c[k] = spread * (-1.0 + (2.0 * k + 1.0) / K);
+    const double tol = 1e-14 / sqrt((double)dim);
+    int it;
+    const int max_it = 200000;
+    for (it = 1; it <= max_it; ++it) {
+        b[0] = -1.0;
+        b[K] = 1.0;
+        for (int k = 1; k < K; ++k) b[k] = 0.5 * (c[k - 1] + c[k]);
+        double delta = 0.0;
+        for (int k = 0; k < K; ++k) {
+            double m0, m1;
+            beta_cell(dim, b[k], b[k + 1], &m0, &m1);
+            const double nc = m1 / m0;
+            const double dd = fabs(nc - c[k]);
+            if (dd > delta) delta = dd;
+            c[k] = nc;
+        }
+        if (delta < tol) break;
+    }
+    if (it > max_it) { free(c); free(b); return -1; }
+    /* the law is symmetric: make the codebook exactly antisymmetric */
+    for (int k = 0; k < K / 2; ++k) {
+        double a = 0.5 * (c[K - 1 - k] - c[k]);
+        c[k] = -a;
+        c[K - 1 - k] = a;
+    }
+    for (int k = 0; k < K; ++k) cents[k] = c[k];
+    for (int k = 1; k < K; ++k) bounds[k - 1] = 0.5 * (c[k - 1] + c[k]);
+    bounds[K / 2 - 1] = 0.0;
+    free(c);
+    free(b);
+    return it;
+}
+
+/* law 0: N(0, 1/dim) (ora_codebook); law 1: the exact Beta law (ora_codebook_beta) */
+int ora_codebook_law(int dim, int bits, int law, double *bounds, double *cents)
+{
+    if (law == 0) return ora_codebook(dim, bits, bounds, cents);
+    if (law == 1) return ora_codebook_beta(dim, bits, bounds, cents);
+    return -1;
+}
+
+/* fp32-rounded codebook of either law */
+int ora_codebook_law_f32(int dim, int bits, int law, float *bounds, float *cents)
+{
+    const int K = 1 << bits;
+    double cb[256], cc[256];
+    int it = ora_codebook_law(dim, bits, law, cb, cc);
+    if (it < 0) return it;
+    for (int k = 0; k < K - 1; ++k) bounds[k] = (float)cb[k];
+    for (int k = 0; k < K; ++k) cents[k] = (float)cc[k];
+    return it;
+}
+
 /* fp32-rounded codebook: the values the quantizer decides against and dequantizes to. */
 int ora_codebook_f32(int dim, int bits, float *bounds, float *cents)
 {
@@ -237,14 +364,14 @@ void ora_unpack_codes(const uint32_t *words, int dim, int beta, int32_t *idx)
  */
 int ora_compress(int is_key, int dim, int bits, int m, const float *R, const float *S,
                  const void *x, int x_is_f16, int64_t n, uint32_t *codes, uint32_t *signs,
-                 uint16_t *norm, uint16_t *rnorm, float *y32_out, float *p32_out)
+                 uint16_t *norm, uint16_t *rnorm, float *y32_out, float *p32_out, int law)
 {
     const int beta = is_key ? bits - 1 : bits;
     if (dim <= 0 || dim % 32 || beta < 1 || beta > 8) return -1;
     if (is_key && (m <= 0 || m % 32)) return -1;
     const int K = 1 << beta;
     float cb32[256], cc32[256];
-    if (ora_codebook_f32(dim, beta, cb32, cc32) < 0) return -1;
+    if (ora_codebook_law_f32(dim, beta, law, cb32, cc32) < 0) return -1;
     const int wpv = beta * dim / 32;
 
 #pragma omp parallel
@@ -336,10 +463,10 @@ static void dequant_one(int dim, int beta, const float *R, const float *cc32, co
 
 /* Dequantize n packed vectors to the original space (TurboQuantMSE.dequantize). */
 int ora_dequantize(int dim, int beta, const float *R, const uint32_t *codes, const uint16_t *norm,
-                   int64_t n, double *out)
+                   int64_t n, double *out, int law)
 {
     float cb32[256], cc32[256];
-    if (ora_codebook_f32(dim, beta, cb32, cc32) < 0) return -1;
+    if (ora_codebook_law_f32(dim, beta, law, cb32, cc32) < 0) return -1;
     const int wpv = beta * dim / 32;
 #pragma omp parallel
     {
@@ -368,13 +495,13 @@ int ora_dequantize(int dim, int beta, const float *R, const uint32_t *codes, con
  */
 int ora_scores(int dim, int bits, int m, const float *R, const float *S, const float *q, int B, int Hq,
                int Hkv, int Nq, int64_t T, const uint32_t *kcodes, const uint32_t *ksigns,
-               const uint16_t *knorm, const uint16_t *krnorm, double *scores)
+               const uint16_t *knorm, const uint16_t *krnorm, double *scores, int law)
 {
     const int beta = bits - 1;
     if (Hkv <= 0 || Hq % Hkv) return -1;
     const int G = Hq / Hkv;
     float cb32[256], cc32[256];
-    if (ora_codebook_f32(dim, beta, cb32, cc32) < 0) return -1;
+    if (ora_codebook_law_f32(dim, beta, law, cb32, cc32) < 0) return -1;
     const int wpk = beta * dim / 32, spk = m / 32;
     const double qjl = sqrt(ORA_PI / 2.0) / (double)m;
     const int64_t slices = (int64_t)B * Hkv;
@@ -439,17 +566,17 @@ int ora_scores(int dim, int bits, int m, const float *R, const float *S, const f
 int ora_attend(int dim, int bits, int m, const float *R, const float *S, const float *q, int B, int Hq,
                int Hkv, int Nq, int64_t T, const uint32_t *kcodes, const uint32_t *ksigns,
                const uint16_t *knorm, const uint16_t *krnorm, const uint32_t *vcodes,
-               const uint16_t *vnorm, double scale, double *out)
+               const uint16_t *vnorm, double scale, double *out, int law)
 {
     if (Hkv <= 0 || Hq % Hkv || T <= 0) return -1;
     const int G = Hq / Hkv;
     const int vbeta = bits;
     float cb32[256], cc32[256];
-    if (ora_codebook_f32(dim, vbeta, cb32, cc32) < 0) return -1;
+    if (ora_codebook_law_f32(dim, vbeta, law, cb32, cc32) < 0) return -1;
     const int wpv = vbeta * dim / 32;
     double *sc = (double *)malloc(sizeof(double) * (size_t)B * Hq * Nq * T);
     if (!sc) return -1;
-    int rc = ora_scores(dim, bits, m, R, S, q, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, sc);
+    int rc = ora_scores(dim, bits, m, R, S, q, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, sc, law);
     if (rc) { free(sc); return rc; }
     const int64_t rows = (int64_t)B * Hq * Nq;
     /* dequantized values of one KV slice, shared by the G heads that read it */

@@ -75,6 +75,24 @@ def test_host_codebook_within_one_ulp_of_oracle(lib, dim, bits):
     np.testing.assert_array_equal(c, -c[::-1])
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("dim", [32, 128, 1024])
+def test_host_beta_codebook_within_one_ulp_of_oracle(lib, dim, bits):
+    # the library's exact-law Lloyd-Max (cumulative table + Hermite interpolation, positive half)
+    # against the oracle's (Gauss-Legendre quadrature in theta, all cells), after fp32 rounding
+    L, _ = lib
+    K = 1 << bits
+    b = np.zeros(K - 1, np.float32)
+    c = np.zeros(K, np.float32)
+    assert L.tq_codebook_beta(dim, bits, b.ctypes.data, c.ctypes.data) == 0
+    ob, oc = oracle.codebook_f32(dim, bits, law="beta")
+    ulp = lambda a, o: np.abs(a.view(np.int32).astype(np.int64) - o.view(np.int32).astype(np.int64))
+    assert ulp(c, oc).max() <= 1
+    assert ulp(b, ob).max() <= 1
+    np.testing.assert_array_equal(c, -c[::-1])
+    assert L.tq_codebook_beta(2, bits, b.ctypes.data, c.ctypes.data) == 1
+
+
 def test_codebook_rejects_bad_args(lib):
     L, _ = lib
     b = np.zeros(16, np.float32)

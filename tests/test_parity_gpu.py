@@ -395,3 +395,42 @@ def test_append_attend(tq, cfg):
                         upto(g["kn"], np.uint16), upto(g["kr"], np.uint16), upto(g["vc"], np.uint32),
                         upto(g["vn"], np.uint16))
     check_close(out, ora, "append + attend")
+
+
+# ------------------------------------------------------- the exact (Beta) coordinate law
+
+@pytest.mark.parametrize("d,bits", [(128, 3), (256, 2), (64, 4)])
+def test_beta_law_compress_scores_attend(tq, d, bits):
+    """Parameter sets prepared with the Beta-law codebooks (tq_prepare_law): compression, scores
+    and attention against the oracle using the same law."""
+    import torch
+    m = d // 2
+    seed = 700 + d + bits
+    R, S = synth.rotation(d, seed), synth.gaussian(m, d, seed + 1)
+    p = tq.Params(d, bits, m, torch.from_numpy(R).cuda(), torch.from_numpy(S).cuda(), law="beta")
+    B, Hkv, G, T = 1, 2, 4, 700
+    x = synth.gaussian(B * Hkv * T, d, seed + 2).astype(np.float16)
+    v = synth.gaussian(B * Hkv * T, d, seed + 3).astype(np.float16)
+    gk = tq.tq_compress_keys(p, torch.from_numpy(x).cuda())
+    gv = tq.tq_compress_values(p, torch.from_numpy(v).cuda())
+    torch.cuda.synchronize()
+    ok = oracle.compress(x, R, S, bits, is_key=True, want_y=True, want_p=True, law="beta")
+    ov = oracle.compress(v, R, None, bits, is_key=False, want_y=True, law="beta")
+    rows = check_codes(gk[0], ok["codes"], ok["y32"], oracle.codebook_f32(d, bits - 1, law="beta")[0], d, bits - 1)
+    check_signs(gk[1], ok["signs"], ok["p32"], m, exempt_rows=rows)
+    check_f16_close(gk[2], ok["norm"], what="norm")
+    check_codes(gv[0], ov["codes"], ov["y32"], oracle.codebook_f32(d, bits, law="beta")[0], d, bits)
+    # scores and attention over the oracle's records (same law on both sides)
+    Hq = Hkv * G
+    q = synth.gaussian(B * Hq, d, seed + 4).reshape(B, Hq, 1, d)
+    qd = torch.from_numpy(q).cuda()
+    kk, vv = _to_dev(ok, ov)
+    s, _, _ = tq.tq_scores(p, qd, kk, Hkv, T)
+    out = tq.tq_attend(p, qd, kk, vv, Hkv, T)
+    torch.cuda.synchronize()
+    ora_s = oracle.scores(q, R, S, bits, B, Hq, Hkv, 1, T, ok["codes"], ok["signs"], ok["norm"], ok["rnorm"],
+                          law="beta")
+    check_close(s, ora_s, "beta-law scores")
+    ora_o = oracle.attend(q, R, S, bits, B, Hq, Hkv, 1, T, ok["codes"], ok["signs"], ok["norm"], ok["rnorm"],
+                          ov["codes"], ov["norm"], law="beta")
+    check_close(out, ora_o, "beta-law attention")
