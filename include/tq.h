@@ -243,6 +243,35 @@ tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new
 tq_status tq_selftest_wait_timeout(int32_t *dev_status, uint32_t timeout_ms, tq_stream_t stream);
 
 /*
+ * Attention over one piece of a longer context, for splitting a long context across GPUs
+ * (nav.superapi.store page, 适用场景: long-context inference; the method's softmax is exact
+ * over any partition of the tokens).  Arguments as tq_attend, with T the tokens of this piece
+ * (records [B, Hkv, T] of this piece only); instead of the output it writes, per query row
+ * [B, Hq, Nq], a partial of dim + 2 floats:
+ *   partial[0]     = M, the largest logit scale * s_t of the piece,
+ *   partial[1]     = l = sum_t e^{scale s_t - M},
+ *   partial[2 + j] = sum_t e^{scale s_t - M} ||v_t|| c[vidx_tj]   (rotated coordinates, unnormalised)
+ *   partial    : device fp32 [B * Hq * Nq, dim + 2]
+ *   scratch    : device, tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, T) bytes
+ */
+tq_status tq_attend_partial(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                            const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                            const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm, float scale,
+                            float *partial, void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                            tq_stream_t stream);
+
+/*
+ * Merge the partials of `parts` pieces of a context (for example gathered from the GPUs that
+ * each attended one piece with tq_attend_partial) into the attention output:
+ *   M = max_k M_k,  out = R^T (sum_k e^{M_k - M} o_k) / (sum_k e^{M_k - M} l_k)
+ *   partials : device fp32 [parts, rows, dim + 2] (piece-major, as an all-gather leaves them)
+ *   out      : device fp32 [rows, dim]   (rows = B * Hq * Nq)
+ * The result equals tq_attend over the whole context up to floating-point rounding.
+ */
+tq_status tq_attend_merge(const tq_params *p, const float *partials, int parts, int64_t rows, float *out,
+                          int32_t *dev_status, tq_stream_t stream);
+
+/*
  * tq_attend_static -- tq_attend for callers that cannot allocate device memory when they call.
  * (The pages have no counterpart: this is an addition of the library.)
  * A serving loop whose device memory is all handed to its own pool up front, or code that must

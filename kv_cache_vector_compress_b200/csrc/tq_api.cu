@@ -283,6 +283,57 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     return from_cuda(e);
 }
 
+tq_status tq_attend_partial(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                            const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                            const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm, float scale,
+                            float *partial, void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                            tq_stream_t stream) {
+    (void)dev_status;
+    tq_status st = check_params(p, true);
+    if (st != TQ_OK) return st;
+    st = check_problem(p, B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm);
+    if (st != TQ_OK) return st;
+    if (!vcodes || !vnorm || !partial || !aligned16(vcodes) || !aligned16(vnorm) || !aligned16(partial))
+        return TQ_ERR_INVALID_ARG;
+    if (!(scale == scale)) return TQ_ERR_INVALID_ARG;  // NaN
+    if (!scratch || !aligned16(scratch)) return TQ_ERR_INVALID_ARG;
+    if (scratch_bytes < tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, T)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm, vcodes, vnorm);
+    if (scale <= 0.f) scale = 1.0f / sqrtf((float)p->dim);
+    cudaStream_t s = (cudaStream_t)stream;
+    float *qprep = (float *)scratch;
+    const AttendPlan plan = plan_attend(P, sp);
+    float *partials = (float *)((char *)scratch + qprep_bytes(P, sp));
+    uint32_t *frag = (uint32_t *)((char *)partials + attend_partials_bytes(P, sp, plan.splits));
+    cudaError_t e = plan.planes ? cudaSuccess : launch_qprep(P, sp, qprep, s);
+    if (e == cudaSuccess) {
+        if (plan.planes) {
+            e = launch_planes(P, sp, scale, frag, plan.pp, true, partial, partials, s, true);
+        } else if (plan.mma) {
+            e = launch_decode_mma(P, sp, qprep, scale, partials, plan.splits, true, s);
+            if (e == cudaSuccess)
+                e = launch_merge_partials(P, (int64_t)B * Hq * Nq, plan.splits, partials,
+                                          (int64_t)plan.splits * (p->dim + 2), p->dim + 2, false, partial, s);
+        } else {
+            e = launch_attend(P, sp, qprep, scale, partials, plan.splits, partial, s, false);
+        }
+    }
+    return from_cuda(e);
+}
+
+tq_status tq_attend_merge(const tq_params *p, const float *partials, int parts, int64_t rows, float *out,
+                          int32_t *dev_status, tq_stream_t stream) {
+    (void)dev_status;
+    tq_status st = check_params(p, false);
+    if (st != TQ_OK) return st;
+    if (parts < 1 || rows < 1) return TQ_ERR_INVALID_ARG;
+    if (!partials || !out || !aligned16(partials) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
+    Prepared P = prepared_view(p);
+    return from_cuda(launch_merge_partials(P, rows, parts, partials, p->dim + 2, rows * (int64_t)(p->dim + 2), true,
+                                           out, (cudaStream_t)stream));
+}
+
 tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new, const void *v_new,
                            tq_dtype dtype, int B, int Hq, int Hkv, int Nq, int64_t t, int64_t t_cap,
                            uint32_t *kcodes, uint32_t *ksigns, uint16_t *knorm, uint16_t *krnorm,

@@ -383,7 +383,7 @@ __host__ __device__ inline PlanesSmem planes_smem(int range, int splits_cap) {
 template <int D, int KB, int VB, bool ATTEND>
 __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
     planes_attend_kernel(Prepared P, ScoreProblem sp, uint32_t *__restrict__ frag, int range, int splits,
-                         float *__restrict__ out, float *__restrict__ partials) {
+                         float *__restrict__ out, float *__restrict__ partials, int merged_partial) {
     using C = PlanesCfg<D, KB, VB>;
     using RG = PlanesRing<D, KB, VB, ATTEND>;
     constexpr int NT = C::NW * 32;
@@ -834,7 +834,8 @@ __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
     if (!last) return;
     __threadfence();
     float *orow = sbuf;                 // [kPRows][D] merged o_rot
-    float *wsp = sbuf + kPRows * D;     // [kPRows][splits] split weights / L
+    float *wsp = sbuf + kPRows * D;     // [kPRows][splits] split weights e^{M_s - M}
+    __shared__ float msh[kPRows], lsh[kPRows];
     for (int r = warp; r < nrows; r += C::NW) {
         const float *pp = partials + qrow_of(r) * splits * (int64_t)(D + 2);
         float M = -INFINITY;
@@ -848,8 +849,10 @@ __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
             Ls = fmaf(w, ps[1], Ls);
         }
         Ls = warp_sum(Ls);
-        __syncwarp();
-        for (int s2 = lane; s2 < splits; s2 += 32) wsp[r * splits + s2] /= Ls;
+        if (lane == 0) {
+            msh[r] = M;
+            lsh[r] = Ls;
+        }
     }
     __syncthreads();
     for (int e = tid; e < nrows * D; e += NT) {
@@ -866,8 +869,20 @@ __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
             for (int u = 0; u < 8; ++u) a8[u] = fmaf(ww[s2 + u], v[u], a8[u]);
         }
         for (; s2 < splits; ++s2) a8[0] = fmaf(ww[s2], pj[(int64_t)s2 * (D + 2)], a8[0]);
-        orow[r * D + j] = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+        const float sum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+        if (merged_partial) {
+            // the slice's partial over its whole context: (M, l, o_rot), unnormalised
+            float *po = out + qrow_of(r) * (int64_t)(D + 2);
+            if (j == 0) {
+                po[0] = msh[r];
+                po[1] = lsh[r];
+            }
+            po[2 + j] = sum;
+        } else {
+            orow[r * D + j] = sum / lsh[r];
+        }
     }
+    if (merged_partial) return;
     __syncthreads();
     for (int j = tid; j < D; j += NT) {
         float a4[kPRows] = {0.f, 0.f, 0.f, 0.f};
@@ -885,7 +900,7 @@ __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
 
 template <int D, int KB, int VB, bool ATTEND>
 cudaError_t launch_planes_t(const Prepared &P, const ScoreProblem &sp, float scale, uint32_t *frag,
-                            int range, int splits, float *out, float *partials, cudaStream_t s) {
+                            int range, int splits, float *out, float *partials, cudaStream_t s, int mp) {
     using C = PlanesCfg<D, KB, VB>;
     const int64_t slices = (int64_t)sp.B * sp.Hkv;
     planes_qfrag_kernel<D, KB><<<(unsigned)slices, 256, 0, s>>>(P, sp, ATTEND ? scale : 1.0f, frag);
@@ -896,22 +911,22 @@ cudaError_t launch_planes_t(const Prepared &P, const ScoreProblem &sp, float sca
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)splits, (unsigned)slices);
-    kern<<<grid, C::NW * 32, L.total, s>>>(P, sp, frag, range, splits, out, partials);
+    kern<<<grid, C::NW * 32, L.total, s>>>(P, sp, frag, range, splits, out, partials, mp);
     return cudaGetLastError();
 }
 
 template <int D, bool ATTEND>
 cudaError_t launch_planes_d(const Prepared &P, const ScoreProblem &sp, float scale, uint32_t *frag, int range,
-                            int splits, float *out, float *partials, cudaStream_t s) {
+                            int splits, float *out, float *partials, cudaStream_t s, int mp) {
     const int kb = P.kbeta, vb = P.vbeta;
     if constexpr (ATTEND) {
-        if (kb == 1 && vb == 2) return launch_planes_t<D, 1, 2, true>(P, sp, scale, frag, range, splits, out, partials, s);
-        if (kb == 2 && vb == 3) return launch_planes_t<D, 2, 3, true>(P, sp, scale, frag, range, splits, out, partials, s);
-        if (kb == 3 && vb == 4) return launch_planes_t<D, 3, 4, true>(P, sp, scale, frag, range, splits, out, partials, s);
+        if (kb == 1 && vb == 2) return launch_planes_t<D, 1, 2, true>(P, sp, scale, frag, range, splits, out, partials, s, mp);
+        if (kb == 2 && vb == 3) return launch_planes_t<D, 2, 3, true>(P, sp, scale, frag, range, splits, out, partials, s, mp);
+        if (kb == 3 && vb == 4) return launch_planes_t<D, 3, 4, true>(P, sp, scale, frag, range, splits, out, partials, s, mp);
     } else {
-        if (kb == 1) return launch_planes_t<D, 1, 2, false>(P, sp, scale, frag, range, splits, out, partials, s);
-        if (kb == 2) return launch_planes_t<D, 2, 2, false>(P, sp, scale, frag, range, splits, out, partials, s);
-        if (kb == 3) return launch_planes_t<D, 3, 2, false>(P, sp, scale, frag, range, splits, out, partials, s);
+        if (kb == 1) return launch_planes_t<D, 1, 2, false>(P, sp, scale, frag, range, splits, out, partials, s, mp);
+        if (kb == 2) return launch_planes_t<D, 2, 2, false>(P, sp, scale, frag, range, splits, out, partials, s, mp);
+        if (kb == 3) return launch_planes_t<D, 3, 2, false>(P, sp, scale, frag, range, splits, out, partials, s, mp);
     }
     return cudaErrorInvalidValue;
 }
@@ -956,17 +971,19 @@ size_t planes_frag_bytes(const Prepared &P, const ScoreProblem &sp) {
 }
 
 cudaError_t launch_planes(const Prepared &P, const ScoreProblem &sp, float scale, uint32_t *frag,
-                          const PlanesPlan &pl, bool attend, float *out, float *partials, cudaStream_t s) {
+                          const PlanesPlan &pl, bool attend, float *out, float *partials, cudaStream_t s,
+                          bool merged_partial) {
+    const int mp = merged_partial ? 1 : 0;
     switch (P.d) {
         case 64:
-            return attend ? launch_planes_d<64, true>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s)
-                          : launch_planes_d<64, false>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s);
+            return attend ? launch_planes_d<64, true>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s, mp)
+                          : launch_planes_d<64, false>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s, mp);
         case 128:
-            return attend ? launch_planes_d<128, true>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s)
-                          : launch_planes_d<128, false>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s);
+            return attend ? launch_planes_d<128, true>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s, mp)
+                          : launch_planes_d<128, false>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s, mp);
         case 256:
-            return attend ? launch_planes_d<256, true>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s)
-                          : launch_planes_d<256, false>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s);
+            return attend ? launch_planes_d<256, true>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s, mp)
+                          : launch_planes_d<256, false>(P, sp, scale, frag, pl.range, pl.splits, out, partials, s, mp);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -164,6 +164,11 @@ int attend_splits(const ScoreProblem &sp);
 size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int splits);
 cudaError_t launch_attend_combine(const Prepared &P, const ScoreProblem &sp, const float *partials, int splits,
                                   float *out, cudaStream_t s);
+// Merge partials (M, l, o_rot) of `parts` context pieces per row: element (row, part) at
+// row * row_stride + part * part_stride.  final: out = R^T o / l [rows, d]; else the merged
+// partial [rows, d + 2].
+cudaError_t launch_merge_partials(const Prepared &P, int64_t rows, int parts, const float *partials,
+                                  int64_t row_stride, int64_t part_stride, bool final, float *out, cudaStream_t s);
 bool decode_mma_supported(const Prepared &P, const ScoreProblem &sp, bool attend);
 int decode_mma_splits(const ScoreProblem &sp);
 cudaError_t launch_decode_mma(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale,
@@ -182,7 +187,8 @@ size_t planes_frag_bytes(const Prepared &P, const ScoreProblem &sp);
 // false: out = scores [B, Hq, Nq, T]) or the attention output (attend = true: out = [B, Hq, Nq, d],
 // through per-range partials [rows, splits, d + 2] that the last CTA of each slice merges).
 cudaError_t launch_planes(const Prepared &P, const ScoreProblem &sp, float scale, uint32_t *frag,
-                          const PlanesPlan &pl, bool attend, float *out, float *partials, cudaStream_t s);
+                          const PlanesPlan &pl, bool attend, float *out, float *partials, cudaStream_t s,
+                          bool merged_partial = false);
 
 // Which attention kernel a problem uses and how many context splits it takes.
 struct AttendPlan {
@@ -230,7 +236,8 @@ cudaError_t launch_scores(const Prepared &P, const ScoreProblem &sp, const float
                           float *scores, cudaStream_t s);
 cudaError_t launch_topk(const ScoreProblem &sp, const float *scores, int topk, int32_t *idx,
                         float *val, cudaStream_t s);
+// final = false: out is the merged partial [rows, d + 2] (max, sum, o_rot) instead of [rows, d]
 cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float *qprep,
-                          float scale, float *partials, int splits, float *out, cudaStream_t s);
+                          float scale, float *partials, int splits, float *out, cudaStream_t s, bool final = true);
 
 }  // namespace tq

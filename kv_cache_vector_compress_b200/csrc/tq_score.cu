@@ -383,59 +383,74 @@ __global__ void __launch_bounds__(kTile) attend_kernel(Prepared P, ScoreProblem 
     (void)rows_total;
 }
 
-// Merge the split-context partials (max, sum, o_rot) of each query row and rotate back:
-// out = R^T (sum_s e^{M_s - M} o_s) / (sum_s e^{M_s - M} l_s).  One block per row; the split loads
-// of a coordinate are issued eight at a time.
-__global__ void __launch_bounds__(128) attend_combine_kernel(Prepared P, int64_t rows, int splits,
+// Merge partials (max M_s, sum l_s, o_s) of each query row: element (row, s) starts at
+// row * row_stride + s * part_stride.  final = true writes out = R^T (sum_s e^{M_s - M} o_s) /
+// (sum_s e^{M_s - M} l_s) [rows, d]; final = false writes the merged partial (M, sum_s e^{M_s - M} l_s,
+// sum_s e^{M_s - M} o_s) [rows, d + 2] in the rotated domain.  One block per row; the loads of a
+// coordinate over the parts are issued eight at a time.
+__global__ void __launch_bounds__(128) attend_combine_kernel(Prepared P, int64_t rows, int parts,
                                                              const float *__restrict__ partials,
+                                                             int64_t row_stride, int64_t part_stride, int final,
                                                              float *__restrict__ out) {
     extern __shared__ float csm[];
     const int d = P.d;
     float *orot = csm;     // [d]
-    float *wts = csm + d;  // [splits]
-    __shared__ float lsum;
+    float *wts = csm + d;  // [parts]
+    __shared__ float lsum, mrow;
     for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
-        const float *pp = partials + row * splits * (int64_t)(d + 2);
+        const float *pp = partials + row * row_stride;
         if (threadIdx.x < 32) {
             const int lane = threadIdx.x;
             float M = -INFINITY;
-            for (int s = lane; s < splits; s += 32) M = fmaxf(M, pp[(int64_t)s * (d + 2)]);
+            for (int s = lane; s < parts; s += 32) M = fmaxf(M, pp[(int64_t)s * part_stride]);
             for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
             float L = 0.f;
-            for (int s = lane; s < splits; s += 32) {
-                const float *ps = pp + (int64_t)s * (d + 2);
+            for (int s = lane; s < parts; s += 32) {
+                const float *ps = pp + (int64_t)s * part_stride;
                 const float w = (ps[0] == -INFINITY) ? 0.f : expf(ps[0] - M);
                 wts[s] = w;
                 L = fmaf(w, ps[1], L);
             }
             for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-            if (lane == 0) lsum = L;
+            if (lane == 0) {
+                lsum = L;
+                mrow = M;
+            }
         }
         __syncthreads();
-        const float invL = 1.f / lsum;
+        const float scl = final ? 1.f / lsum : 1.f;
         for (int j = threadIdx.x; j < d; j += blockDim.x) {
             const float *pj = pp + 2 + j;
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             int s = 0;
-            for (; s + 8 <= splits; s += 8) {
+            for (; s + 8 <= parts; s += 8) {
                 float v[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = pj[(int64_t)(s + u) * (d + 2)];
+                for (int u = 0; u < 8; ++u) v[u] = pj[(int64_t)(s + u) * part_stride];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) acc[u] = fmaf(wts[s + u], v[u], acc[u]);
             }
-            for (; s < splits; ++s) acc[0] = fmaf(wts[s], pj[(int64_t)s * (d + 2)], acc[0]);
-            orot[j] = (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]))) * invL;
+            for (; s < parts; ++s) acc[0] = fmaf(wts[s], pj[(int64_t)s * part_stride], acc[0]);
+            orot[j] = (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]))) * scl;
         }
         __syncthreads();
-        for (int j = threadIdx.x; j < d; j += blockDim.x) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (final) {
+            for (int j = threadIdx.x; j < d; j += blockDim.x) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-            for (int i = 0; i < d; i += 4) {
+                for (int i = 0; i < d; i += 4) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) acc[u] = fmaf(P.R[(int64_t)(i + u) * d + j], orot[i + u], acc[u]);
+                    for (int u = 0; u < 4; ++u) acc[u] = fmaf(P.R[(int64_t)(i + u) * d + j], orot[i + u], acc[u]);
+                }
+                out[row * d + j] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
-            out[row * d + j] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        } else {
+            float *po = out + row * (int64_t)(d + 2);
+            if (threadIdx.x == 0) {
+                po[0] = mrow;
+                po[1] = lsum;
+            }
+            for (int j = threadIdx.x; j < d; j += blockDim.x) po[2 + j] = orot[j];
         }
         __syncthreads();
     }
@@ -503,7 +518,7 @@ static cudaError_t launch_attend_cpt(const Prepared &P, const ScoreProblem &sp, 
 }
 
 cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float *qprep, float scale,
-                          float *partials, int splits, float *out, cudaStream_t s) {
+                          float *partials, int splits, float *out, cudaStream_t s, bool final) {
     cudaError_t e;
     const int cpt = (P.d + kTile - 1) / kTile;
     switch (cpt) {
@@ -514,21 +529,30 @@ cudaError_t launch_attend(const Prepared &P, const ScoreProblem &sp, const float
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
+    if (!final)
+        return launch_merge_partials(P, (int64_t)sp.B * sp.Hq * sp.Nq, splits, partials, (int64_t)splits * (P.d + 2),
+                                     P.d + 2, false, out, s);
     return launch_attend_combine(P, sp, partials, splits, out, s);
 }
 
-cudaError_t launch_attend_combine(const Prepared &P, const ScoreProblem &sp, const float *partials, int splits,
-                                  float *out, cudaStream_t s) {
-    const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
+cudaError_t launch_merge_partials(const Prepared &P, int64_t rows, int parts, const float *partials,
+                                  int64_t row_stride, int64_t part_stride, bool final, float *out, cudaStream_t s) {
     const int blocks = (int)(rows < 148 * 16 ? rows : 148 * 16);
-    const size_t smem = sizeof(float) * ((size_t)P.d + (size_t)splits);
+    const size_t smem = sizeof(float) * ((size_t)P.d + (size_t)parts);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
-    attend_combine_kernel<<<blocks, 128, smem, s>>>(P, rows, splits, partials, out);
+    attend_combine_kernel<<<blocks, 128, smem, s>>>(P, rows, parts, partials, row_stride, part_stride, final ? 1 : 0,
+                                                    out);
     return cudaGetLastError();
+}
+
+cudaError_t launch_attend_combine(const Prepared &P, const ScoreProblem &sp, const float *partials, int splits,
+                                  float *out, cudaStream_t s) {
+    const int64_t rows = (int64_t)sp.B * sp.Hq * sp.Nq;
+    return launch_merge_partials(P, rows, splits, partials, (int64_t)splits * (P.d + 2), P.d + 2, true, out, s);
 }
 
 }  // namespace tq

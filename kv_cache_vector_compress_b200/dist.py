@@ -2,9 +2,11 @@
 
 The compression path partitions into independent (batch, KV-head) slices, so ranks share no data
 and no collective runs on the data path; the timing reduction (the reported time of a timed
-region is the maximum over ranks) is the only collective there.  Vector search over a database
-sharded across ranks has one real exchange: every rank's top-k list of each query is gathered and
-merged (sharded_topk).
+region is the maximum over ranks) is the only collective there.  Two paths have one real exchange
+each: vector search over a database sharded across ranks gathers every rank's top-k list of each
+query and merges them (sharded_topk); attention over one long context split across ranks gathers
+each rank's (max, sum, weighted value sum) partial of its token range and merges them
+(sharded_attend).
 """
 from __future__ import annotations
 
@@ -91,6 +93,34 @@ def sharded_topk(local_idx: torch.Tensor, local_val: torch.Tensor, k: int, offse
     dist.all_gather(all_v, local_val.contiguous())
     dist.all_gather(all_i, gidx.contiguous())
     return merge_topk(torch.cat(all_v, dim=-1), torch.cat(all_i, dim=-1), k)
+
+
+def context_shard(T: int, world: int, rank: int) -> tuple[int, int]:
+    """Contiguous token range [start, start + count) of a T-token context that this rank attends
+    when one long context is split across the ranks."""
+    return shard(T, world, rank)
+
+
+def gather_partials(partial: torch.Tensor) -> torch.Tensor:
+    """All ranks' attention partials [..., dim + 2] stacked in rank order: [world, ...] (one
+    all_gather; every rank receives all of them)."""
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return partial.unsqueeze(0)
+    world = dist.get_world_size()
+    parts = [torch.empty_like(partial) for _ in range(world)]
+    dist.all_gather(parts, partial.contiguous())
+    return torch.stack(parts)
+
+
+def sharded_attend(p, q: torch.Tensor, keys, values, Hkv: int, T_local: int, scale: float = 0.0):
+    """Attention over a long context split across the ranks: every rank holds the packed keys and
+    values of its own token range (context_shard) and the same queries; it computes the partial of
+    its range (tq_attend_partial), the partials are all-gathered, and each rank merges them
+    (tq_attend_merge: log-sum-exp of the pieces, then the single rotation back).  Returns the
+    attention output [B, Hq, Nq, dim] on every rank."""
+    from . import tq
+    part = tq.tq_attend_partial(p, q, keys, values, Hkv, T_local, scale=scale)
+    return tq.tq_attend_merge(p, gather_partials(part))
 
 
 def destroy():

@@ -69,6 +69,11 @@ _lib.tq_attend.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P
                            _SZ, _P, _P]
 _lib.tq_attend.restype = _I
 
+_lib.tq_attend_partial.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
+                                   _SZ, _P, _P]
+_lib.tq_attend_partial.restype = _I
+_lib.tq_attend_merge.argtypes = [_PP, _P, _I, _I64, _P, _P, _P]
+_lib.tq_attend_merge.restype = _I
 _lib.tq_attend_static.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P,
                                   _P, _P]
 _lib.tq_attend_static.restype = _I
@@ -83,7 +88,8 @@ LAWS = {"gaussian": TQ_LAW_GAUSSIAN, "beta": TQ_LAW_BETA}
 EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_codebook_beta", "tq_workspace_bytes",
            "tq_prepare", "tq_prepare_law",
            "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores",
-           "tq_attend_scratch_bytes", "tq_attend", "tq_append_attend", "tq_selftest_wait_timeout",
+           "tq_attend_scratch_bytes", "tq_attend", "tq_attend_partial", "tq_attend_merge", "tq_append_attend",
+           "tq_selftest_wait_timeout",
            "tq_attend_static"]
 
 
@@ -286,6 +292,38 @@ def tq_append_attend(p: Params, q: torch.Tensor, k_new: torch.Tensor, v_new: tor
                                  _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr), _ptr(vc), _ptr(vn), float(scale),
                                  _ptr(out), _ptr(scratch), scratch.numel(), _ptr(dev_status), _stream()),
            "tq_append_attend")
+    return out
+
+
+def tq_attend_partial(p: Params, q: torch.Tensor, keys, values, Hkv: int, T: int, scale: float = 0.0,
+                      partial=None, scratch=None, dev_status=None):
+    """Attention partial over one piece of a context: [B, Hq, Nq, dim + 2] fp32 holding, per query
+    row, the piece's largest logit, the sum of e^(logit - max), and the unnormalised rotated
+    weighted value sum (see tq_attend_merge)."""
+    B, Hq, Nq, d = q.shape
+    kc, ks, kn, kr = keys
+    vc, vn = values
+    dev = q.device
+    if partial is None:
+        partial = torch.empty((B, Hq, Nq, d + 2), dtype=torch.float32, device=dev)
+    if scratch is None:
+        scratch = torch.empty(max(tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, T), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.tq_attend_partial(p.ref, _ptr(q), B, Hq, Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr),
+                                  _ptr(vc), _ptr(vn), float(scale), _ptr(partial), _ptr(scratch), scratch.numel(),
+                                  _ptr(dev_status), _stream()), "tq_attend_partial")
+    return partial
+
+
+def tq_attend_merge(p: Params, partials: torch.Tensor, out=None, dev_status=None):
+    """Merge partials [parts, B, Hq, Nq, dim + 2] of the pieces of one context into the attention
+    output [B, Hq, Nq, dim]."""
+    parts = partials.shape[0]
+    shape = partials.shape[1:-1]
+    rows = int(torch.tensor(shape).prod().item()) if len(shape) else 1
+    if out is None:
+        out = torch.empty((*shape, p.dim), dtype=torch.float32, device=partials.device)
+    _check(_lib.tq_attend_merge(p.ref, _ptr(partials), parts, rows, _ptr(out), _ptr(dev_status), _stream()),
+           "tq_attend_merge")
     return out
 
 

@@ -434,3 +434,43 @@ def test_beta_law_compress_scores_attend(tq, d, bits):
     ora_o = oracle.attend(q, R, S, bits, B, Hq, Hkv, 1, T, ok["codes"], ok["signs"], ok["norm"], ok["rnorm"],
                           ov["codes"], ov["norm"], law="beta")
     check_close(out, ora_o, "beta-law attention")
+
+
+# ------------------------------------------- one long context split into pieces (multi-GPU)
+
+@pytest.mark.parametrize("cfg", [
+    dict(d=128, m=64, bits=3, B=2, Hkv=2, G=4, Nq=1, cuts=(0, 1000, 2100, 3000)),  # bit-plane kernel
+    dict(d=256, m=128, bits=2, B=1, Hkv=1, G=4, Nq=1, cuts=(0, 1, 700)),          # a one-token piece
+    dict(d=64, m=32, bits=4, B=1, Hkv=2, G=1, Nq=9, cuts=(0, 129, 400)),          # register-MMA kernel
+    dict(d=32, m=32, bits=3, B=1, Hkv=1, G=2, Nq=1, cuts=(0, 60, 61, 127)),       # CUDA-core kernel
+])
+def test_context_pieces_merge_to_whole_attention(tq, cfg):
+    """The context of every (batch, KV head) cut into pieces, as ranks that each hold one token
+    range would hold them: tq_attend_partial on each piece, tq_attend_merge of the stacked
+    partials, against the oracle's attention over the whole context."""
+    import torch
+    c = cfg
+    cuts = c["cuts"]
+    T = cuts[-1]
+    R, S, k, v = _oracle_cache(900 + c["d"] + T, c["d"], c["m"], c["bits"], c["B"], c["Hkv"], T)
+    Hq = c["Hkv"] * c["G"]
+    q = synth.gaussian(c["B"] * Hq * c["Nq"], c["d"], 19).reshape(c["B"], Hq, c["Nq"], c["d"])
+    ora = oracle.attend(q, R, S, c["bits"], c["B"], Hq, c["Hkv"], c["Nq"], T, k["codes"], k["signs"], k["norm"],
+                        k["rnorm"], v["codes"], v["norm"])
+    p = _params(tq, R, S, c["bits"], c["m"])
+    qd = torch.from_numpy(q).cuda()
+    nsl = c["B"] * c["Hkv"]
+
+    def piece(a, t0, t1):
+        return np.ascontiguousarray(a.reshape(nsl, T, -1)[:, t0:t1]).reshape(nsl * (t1 - t0), -1)
+
+    parts = []
+    for t0, t1 in zip(cuts[:-1], cuts[1:]):
+        kp = {n: piece(k[n], t0, t1) for n in ("codes", "signs")}
+        kp.update({n: piece(k[n].reshape(-1, 1), t0, t1).reshape(-1) for n in ("norm", "rnorm")})
+        vp = {"codes": piece(v["codes"], t0, t1), "norm": piece(v["norm"].reshape(-1, 1), t0, t1).reshape(-1)}
+        kk, vv = _to_dev(kp, vp)
+        parts.append(tq.tq_attend_partial(p, qd, kk, vv, c["Hkv"], t1 - t0))
+    out = tq.tq_attend_merge(p, torch.stack(parts))
+    torch.cuda.synchronize()
+    check_close(out, ora, "merged context pieces")
