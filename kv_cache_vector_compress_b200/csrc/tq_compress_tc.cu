@@ -5,14 +5,15 @@
 //   rotation    ACC[v, j] = sum_i X[v, i] (R_hi + R_lo)[j, i]          tcgen05, smem x smem
 //               (X is the fp16 input tile, exact in fp16; R * 2^8 = R_hi + R_lo in fp16, so
 //               the product carries ~22 bits of R and the accumulator is fp32)
-//   code step   n = ||x|| (from the input tile), y = ACC / (2^8 n), idx = code of y, planar pack;
+//   code step   n = ||R x|| = ||ACC|| / 2^8 (the two halves of a row summed by its two threads),
+//               y = ACC / (2^8 n), idx = code of y, planar pack;
 //               keys: e = 2^14 (y - c[idx]) split into fp16 hi + lo, written back into TMEM
 //   projection  P[v, a] = sum_j (E_hi (S'_hi + S'_lo) + E_lo S'_hi)[v, j]   tcgen05, tmem x smem
 //               with S' = S R^T, so P is a positive multiple of S r for the residual r = R^T e;
 //   sign step   QJL sign bits of P.
-// One thread owns one vector (one TMEM lane) and half of its coordinates.  Warp roles: warp 0
-// loads (TMA) and owns TMEM, warp 1 issues the MMAs, warps 2..9 run the code and sign steps of
-// every tile, warps 10..11 take the row norms.  TMEM holds up to four rotation accumulators
+// One thread owns one vector (one TMEM lane) and half of its coordinates.  Warp roles (10 warps):
+// warp 0 loads (TMA) and owns TMEM, warp 1 issues the MMAs, warps 2..9 run the norm, code and
+// sign steps of every tile.  TMEM holds up to four rotation accumulators
 // (keys: three beside two projection accumulators), so the rotation of later tiles and the
 // projection of earlier ones keep the tensor cores busy while a tile is being coded.
 #include <cudaTypedefs.h>
@@ -79,7 +80,7 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int m, bool is_key) {
 enum BarIdx {
     kOpnd = 0,
     kFull = 1,       // [4] input stage landed
-    kEmpty = 5,      // [4] input stage consumed (rotation + both norm warps)
+    kEmpty = 5,      // [4] input stage consumed (its rotation MMAs completed)
     kRotFull = 9,    // [4] rotation accumulator ready
     kEReady = 13,    // [4] codes written; keys: residual in TMEM; values: accumulator free
     kNormReady = 17, // [4] both halves' squared row norms of the slot's tile
