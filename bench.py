@@ -523,6 +523,18 @@ def run_workload(args):
         r["tflops_mma"] = 2.0 * pad(Nq) * pad(N) * (3 * d + 2 * m) / (ms * 1e-3) / 1e12
         r["frac_tensor"] = r["tflops_mma"] / (ri.world * pk["bf16_tflops"]) if pk.get("bf16_tflops") else None
         out.append(r)
+
+        # tq_search: the same launch with single fp16 operand products (one per column)
+        def search16():
+            tq.tq_search(p, Qv, keys, 1, Nl, want_scores=False, topk=k, topk_idx=ti, topk_val=tv, scratch=scr)
+            if ri.world > 1:
+                tqdist.sharded_topk(ti.view(Nq, k), tv.view(Nq, k), k, start)
+        ms = timed_ranks(search16, steps=5, warmup=3)
+        r = rec("search_top10_fp16", ms, N * Nq, "query_key_pairs", N * kb, gpus=ri.world)
+        r["tflops_equiv"] = 2.0 * Nq * N * (d + m) / (ms * 1e-3) / 1e12
+        r["tflops_mma"] = 2.0 * pad(Nq) * pad(N) * (d + m) / (ms * 1e-3) / 1e12
+        r["frac_tensor"] = r["tflops_mma"] / (ri.world * pk["bf16_tflops"]) if pk.get("bf16_tflops") else None
+        out.append(r)
         name = (f"vector search: {N} x d1024 4-bit Prod (m=512) fp32 DB, 1024 queries, top-10"
                 + (f", sharded over {ri.world} GPUs (per-rank top-k lists gathered and merged)" if ri.world > 1 else ""))
     elif wl == 6:

@@ -182,6 +182,24 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
                     tq_stream_t stream);
 
 /*
+ * tq_search -- tq_scores for vector-database search ("TurboQuant er nå tilgjengelig som
+ * Python-bibliotek", jansverre.net, "Hvem er dette nyttig for?": nearest-neighbour search over
+ * compressed vectors), with the tensor-core products taken on single fp16 operands.
+ * Arguments, layouts, scratch size (tq_scores_scratch_bytes), ownership and errors are those of
+ * tq_scores.  Where the tensor-core search path runs (more than 64 query rows per KV head,
+ * dim and proj_dim multiples of 64, 2-4 bit keys) each operand of a product is the fp16
+ * rounding of its exact value (relative 2^-11), so a score differs from the exact estimator by at
+ * most 2^-10 ||k|| (sum_i |q_rot,i c_i| + rho sqrt(pi/2)/m sum_j |(S q)_j|) beyond fp32
+ * accumulation; with unit queries and keys at dim 1024 the typical difference is about 1e-5.
+ * Other shapes run exactly as tq_scores.  The top-k is the k best of these scores.
+ */
+tq_status tq_search(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx,
+                    float *topk_val, void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                    tq_stream_t stream);
+
+/*
  * Attention over a compressed cache, fused: scores from the packed keys, softmax of
  * scale*scores over all T tokens (no mask), weighted sum of the dequantized values
  * (nav.superapi.store page, 常见使用模式: "softmax 后对解压的值做加权求和"):

@@ -189,10 +189,12 @@ size_t tq_scores_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int N
     return bytes;
 }
 
-tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
-                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
-                    const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx, float *topk_val,
-                    void *scratch, size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
+namespace {
+tq_status scores_impl(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                      const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                      const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx, float *topk_val,
+                      void *scratch, size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream,
+                      bool fp16) {
     tq_status st = check_params(p, true);
     if (st != TQ_OK) return st;
     st = check_problem(p, B, Hq, Hkv, Nq, T, q, kcodes, ksigns, knorm, krnorm);
@@ -220,11 +222,11 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     cudaError_t e = plan.planes ? cudaSuccess : launch_qprep(P, sp, qprep, s);
     if (e != cudaSuccess) return from_cuda(e);
     if (plan.fused_topk) {
-        e = launch_search(P, sp, qprep, search_scratch, scores, topk, topk_idx, topk_val, dev_status, s);
+        e = launch_search(P, sp, qprep, search_scratch, scores, topk, topk_idx, topk_val, dev_status, s, fp16);
         return from_cuda(e);
     }
     if (plan.search)
-        e = launch_search(P, sp, qprep, search_scratch, sbuf, 0, nullptr, nullptr, dev_status, s);
+        e = launch_search(P, sp, qprep, search_scratch, sbuf, 0, nullptr, nullptr, dev_status, s, fp16);
     else if (plan.planes)
         e = launch_planes(P, sp, 1.0f, frag, plan_planes(sp), false, sbuf, nullptr, s);
     else if (plan.mma)
@@ -233,6 +235,23 @@ tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
         e = launch_scores(P, sp, qprep, sbuf, s);
     if (e == cudaSuccess && topk > 0) e = launch_topk(sp, sbuf, topk, topk_idx, topk_val, s);
     return from_cuda(e);
+}
+}  // namespace
+
+tq_status tq_scores(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx, float *topk_val,
+                    void *scratch, size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
+    return scores_impl(p, q, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, scores, topk, topk_idx, topk_val,
+                       scratch, scratch_bytes, dev_status, stream, false);
+}
+
+tq_status tq_search(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
+                    const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
+                    const uint16_t *krnorm, float *scores, int topk, int32_t *topk_idx, float *topk_val,
+                    void *scratch, size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
+    return scores_impl(p, q, B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, scores, topk, topk_idx, topk_val,
+                       scratch, scratch_bytes, dev_status, stream, true);
 }
 
 size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T) {

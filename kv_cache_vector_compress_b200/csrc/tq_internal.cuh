@@ -210,9 +210,10 @@ size_t topk_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
 // Many query rows per (batch, KV head): tensor-core scores with an optional fused top-k.
 bool search_tc_supported(const Prepared &P, const ScoreProblem &sp, int topk);
 size_t search_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk);
+// fp16: single fp16 operand products (tq_search) instead of the hi + lo splits (tq_scores)
 cudaError_t launch_search(const Prepared &P, const ScoreProblem &sp, const float *qprep, void *scratch,
                           float *scores, int topk, int32_t *topk_idx, float *topk_val, int32_t *dev_status,
-                          cudaStream_t s);
+                          cudaStream_t s, bool fp16 = false);
 
 // Which kernels tq_scores runs: the tensor-core search (top-k fused when short enough), the
 // register-MMA decode kernel (few rows), or the plain kernel; a separate top-k pass otherwise.

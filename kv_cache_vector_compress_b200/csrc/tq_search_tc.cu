@@ -15,6 +15,9 @@
 // accumulator slots let the epilogue of one tile overlap the MMAs of the next; it transposes the
 // scores through shared memory and keeps running per-row top-k lists, merged by a small kernel.
 // Every operand product is exact in fp32 up to the dropped lo x lo terms (relative 2^-22).
+// The single-product form (FP16 = true, tq_search) keeps only the hi x hi products: every operand
+// is rounded to fp16 once (relative 2^-11), so a score moves by at most
+// 2^-10 ||k|| (sum_i |q_rot,i c_i| + rho gamma sum_j |(S q)_j|) from the exact one.
 #include <math.h>
 
 #include "tq_common.cuh"
@@ -217,7 +220,7 @@ __device__ __forceinline__ bool search_better(float va, int32_t ia, float vb, in
 }
 
 
-template <int KB>
+template <int KB, bool FP16>
 __global__ void __launch_bounds__(kSThreads, 1)
     search_gemm_kernel(Prepared P, ScoreProblem sp, SearchGeom g, const uint8_t *__restrict__ qsw,
                        const int *__restrict__ uexp, float *__restrict__ scores, int K, float *__restrict__ cand_v,
@@ -304,8 +307,10 @@ __global__ void __launch_bounds__(kSThreads, 1)
             for (int gk = 0; gk < total; ++gk) {
                 const int st = gk % kSStages;
                 if (gk >= kSStages && !mbar_wait(&bars[kSEmpty + st], ((gk / kSStages) - 1) & 1, abort_s)) break;
-                mbar_arrive_expect_tx(&bars[kBFull + st], kStageBytes);
-                bulk_load(sm + L.stage + st * kStageBytes, qsw_u + (size_t)(gk % NKB) * kStageBytes, kStageBytes,
+                // the single-product form reads only the hi half of a B tile
+                constexpr uint32_t kCopy = FP16 ? kBTile : kStageBytes;
+                mbar_arrive_expect_tx(&bars[kBFull + st], kCopy);
+                bulk_load(sm + L.stage + st * kStageBytes, qsw_u + (size_t)(gk % NKB) * kStageBytes, kCopy,
                           &bars[kBFull + st]);
                 issued = gk + 1;
             }
@@ -341,8 +346,10 @@ __global__ void __launch_bounds__(kSThreads, 1)
                         const uint32_t a_hi = a0 + 32 * (k >> 1) + 8 * (k & 1);
                         const uint64_t dh = sdesc_sw128(b_hi + 32 * k), dl = sdesc_sw128(b_lo + 32 * k);
                         mma_ts(acc, a_hi, dh, idesc, (kbi | k) ? 1u : 0u);
-                        mma_ts(acc, a_hi, dl, idesc, 1u);
-                        if (cen) mma_ts(acc, a_hi + 16, dh, idesc, 1u);
+                        if constexpr (!FP16) {
+                            mma_ts(acc, a_hi, dl, idesc, 1u);
+                            if (cen) mma_ts(acc, a_hi + 16, dh, idesc, 1u);
+                        }
                     }
                     mma_commit(&bars[kSEmpty + st]);
                 }
@@ -425,7 +432,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
                         for (int q = 0; q < 16; ++q) hp[q] = lp[q] = 0u;
                     }
                     tmem_st16(ta + 32 * h, hp);
-                    tmem_st16(ta + 32 * h + 16, lp);
+                    if constexpr (!FP16) tmem_st16(ta + 32 * h + 16, lp);
                 }
             } else {
                 // projections 64 (kbi - DKB) + 32 h + (0..31): +-rho 2^eA, sign bit set = +1
@@ -703,13 +710,13 @@ __global__ void search_merge_kernel(ScoreProblem sp, SearchGeom g, int K, const 
     }
 }
 
-template <int KB>
+template <int KB, bool FP16>
 cudaError_t launch_search_kb(const Prepared &P, const ScoreProblem &sp, const SearchGeom &g, const uint8_t *qsw,
                              const int *uexp, float *scores, int K, float *cv, int32_t *ci, int32_t *dev_status,
                              cudaStream_t s) {
     const SearchSmem L = search_smem_layout(K, KB);
     const size_t smem = L.total + 1024;
-    auto kern = search_gemm_kernel<KB>;
+    auto kern = search_gemm_kernel<KB, FP16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<g.units * g.kc, kSThreads, smem, s>>>(P, sp, g, qsw, uexp, scores, K, cv, ci, dev_status);
@@ -753,7 +760,7 @@ size_t search_scratch_bytes(const Prepared &P, const ScoreProblem &sp, int topk)
 
 cudaError_t launch_search(const Prepared &P, const ScoreProblem &sp, const float *qprep, void *scratch,
                           float *scores, int topk, int32_t *topk_idx, float *topk_val, int32_t *dev_status,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool fp16) {
     const SearchGeom g = search_geom(P, sp);
     const SearchScratch S = search_scratch_layout(g, topk);
     uint8_t *base = (uint8_t *)scratch;
@@ -768,10 +775,13 @@ cudaError_t launch_search(const Prepared &P, const ScoreProblem &sp, const float
     search_tiles_kernel<<<dim3((unsigned)g.units, (unsigned)g.nkb), 256, 0, s>>>(P, sp, g, qprep, umax, qsw, uexp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    switch (P.kbeta) {
-        case 1: e = launch_search_kb<1>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
-        case 2: e = launch_search_kb<2>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
-        case 3: e = launch_search_kb<3>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
+    switch (P.kbeta * 2 + (fp16 ? 1 : 0)) {
+        case 2: e = launch_search_kb<1, false>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
+        case 3: e = launch_search_kb<1, true>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
+        case 4: e = launch_search_kb<2, false>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
+        case 5: e = launch_search_kb<2, true>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
+        case 6: e = launch_search_kb<3, false>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
+        case 7: e = launch_search_kb<3, true>(P, sp, g, qsw, uexp, scores, topk, cv, ci, dev_status, s); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess || topk == 0) return e;

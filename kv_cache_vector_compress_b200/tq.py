@@ -60,6 +60,8 @@ _lib.tq_scores_scratch_bytes.argtypes = [_PP, _I, _I, _I, _I, _I64, _I]
 _lib.tq_scores_scratch_bytes.restype = _SZ
 _lib.tq_scores.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P, _P]
 _lib.tq_scores.restype = _I
+_lib.tq_search.argtypes = _lib.tq_scores.argtypes
+_lib.tq_search.restype = _I
 _lib.tq_append_attend.argtypes = [_PP, _P, _P, _P, _I, _I, _I, _I, _I, _I64, _I64, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_float, _P, _P, _SZ, _P, _P]
 _lib.tq_append_attend.restype = _I
@@ -87,7 +89,7 @@ LAWS = {"gaussian": TQ_LAW_GAUSSIAN, "beta": TQ_LAW_BETA}
 
 EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_codebook_beta", "tq_workspace_bytes",
            "tq_prepare", "tq_prepare_law",
-           "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores",
+           "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores", "tq_search",
            "tq_attend_scratch_bytes", "tq_attend", "tq_attend_partial", "tq_attend_merge", "tq_append_attend",
            "tq_selftest_wait_timeout",
            "tq_attend_static"]
@@ -226,7 +228,7 @@ def tq_scores_scratch_bytes(p: Params, B, Hq, Hkv, Nq, T, topk=0) -> int:
 
 
 def tq_scores(p: Params, q: torch.Tensor, keys, Hkv: int, T: int, want_scores: bool = True, topk: int = 0,
-              scores=None, topk_idx=None, topk_val=None, scratch=None, dev_status=None):
+              scores=None, topk_idx=None, topk_val=None, scratch=None, dev_status=None, _fn="tq_scores"):
     """Scores [B, Hq, Nq, T] (fp32) of queries q [B, Hq, Nq, dim] against packed keys
     (codes, signs, norm, rnorm) laid out [B, Hkv, T].  With topk > 0 also returns the top-k
     indices and values per row.  Returns (scores or None, topk_idx or None, topk_val or None)."""
@@ -243,10 +245,18 @@ def tq_scores(p: Params, q: torch.Tensor, keys, Hkv: int, T: int, want_scores: b
     need = tq_scores_scratch_bytes(p, B, Hq, Hkv, Nq, T, topk)
     if scratch is None:
         scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    _check(_lib.tq_scores(p.ref, _ptr(q), B, Hq, Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr),
-                          _ptr(scores) if want_scores else None, topk, _ptr(topk_idx), _ptr(topk_val),
-                          _ptr(scratch), scratch.numel(), _ptr(dev_status), _stream()), "tq_scores")
+    _check(getattr(_lib, _fn)(p.ref, _ptr(q), B, Hq, Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr),
+                              _ptr(scores) if want_scores else None, topk, _ptr(topk_idx), _ptr(topk_val),
+                              _ptr(scratch), scratch.numel(), _ptr(dev_status), _stream()), _fn)
     return scores, topk_idx, topk_val
+
+
+def tq_search(p: Params, q: torch.Tensor, keys, Hkv: int, T: int, want_scores: bool = True, topk: int = 0,
+              scores=None, topk_idx=None, topk_val=None, scratch=None, dev_status=None):
+    """tq_scores with single fp16 operand products on the tensor-core search path (vector
+    search; the score error bound is stated in the C header).  Same arguments and results."""
+    return tq_scores(p, q, keys, Hkv, T, want_scores, topk, scores, topk_idx, topk_val, scratch, dev_status,
+                     _fn="tq_search")
 
 
 def tq_attend_scratch_bytes(p: Params, B, Hq, Hkv, Nq, T) -> int:

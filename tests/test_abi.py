@@ -155,15 +155,17 @@ def test_argument_errors_return_before_any_launch(lib):
                             ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
-    call = lambda B, Hq, Hkv, Nq, T, topk=0, sc=fake, sb=1 << 40: L.tq_scores(
-        P(good), fake, B, Hq, Hkv, Nq, T, fake, fake, fake, fake, sc, topk, fake, fake, fake, sb, None, None)
-    assert call(1, 3, 2, 1, 10) == 1      # Hq not a multiple of Hkv
-    assert call(1, 4, 2, 1, 0) == 1       # empty cache
-    assert call(1, 4, 2, 0, 10) == 1      # no queries
-    assert call(1, 4, 2, 1, 10, topk=11) == 1  # topk > T
-    assert call(1, 4, 2, 1, 100, topk=65) == 1  # topk above the maximum
-    assert call(1, 4, 2, 1, 10, sc=None) == 1  # nothing to return
-    assert call(1, 4, 2, 1, 10, sb=0) == 1  # scratch too small
+    L.tq_search.argtypes = L.tq_scores.argtypes
+    for fn in (L.tq_scores, L.tq_search):  # tq_search takes tq_scores' arguments and checks
+        call = lambda B, Hq, Hkv, Nq, T, topk=0, sc=fake, sb=1 << 40: fn(
+            P(good), fake, B, Hq, Hkv, Nq, T, fake, fake, fake, fake, sc, topk, fake, fake, fake, sb, None, None)
+        assert call(1, 3, 2, 1, 10) == 1      # Hq not a multiple of Hkv
+        assert call(1, 4, 2, 1, 0) == 1       # empty cache
+        assert call(1, 4, 2, 0, 10) == 1      # no queries
+        assert call(1, 4, 2, 1, 10, topk=11) == 1  # topk > T
+        assert call(1, 4, 2, 1, 100, topk=65) == 1  # topk above the maximum
+        assert call(1, 4, 2, 1, 10, sc=None) == 1  # nothing to return
+        assert call(1, 4, 2, 1, 10, sb=0) == 1  # scratch too small
     L.tq_attend.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,

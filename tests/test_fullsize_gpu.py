@@ -174,6 +174,16 @@ def test_workload5_vector_search(tq):
     keep = np.array([i for i in range(len(rows)) if i not in bad])
     g = sc[0, 0, :16][:, torch.from_numpy(rows[keep]).cuda()].cpu().numpy()
     check_close(g, ora[0, 0][:, keep], "sampled scores")
+    # the fp16-operand search (the launch the vector-search benchmark times) on the same keys
+    sc16, ti16, tv16 = tq.tq_search(p, Q, keys, 1, N, want_scores=True, topk=k)
+    torch.cuda.synchronize()
+    g16 = sc16[0, 0, :16][:, torch.from_numpy(rows[keep]).cuda()].cpu().numpy()
+    check_close(g16, ora[0, 0][:, keep], "sampled fp16-operand scores")
+    for r in range(0, Nq, 97):
+        row = sc16[0, 0, r].cpu().numpy().astype(np.float64)
+        order = np.lexsort((np.arange(N), -row))[:k]
+        np.testing.assert_array_equal(ti16[0, 0, r].cpu().numpy(), order)
+    del sc16
     # top-k is exactly the k best of the returned scores (value desc, index asc)
     for r in range(0, Nq, 97):
         row = sc[0, 0, r].cpu().numpy().astype(np.float64)
@@ -183,9 +193,9 @@ def test_workload5_vector_search(tq):
 
 
 def test_workload5_topk_against_oracle(tq):
-    """The vector-search launch (1M packed keys, d=1024, 4-bit, 1024 query rows, top-10 fused into
-    the search kernel) against the oracle's exact top-10 over the whole database, for 8 of the
-    query rows.  Both sides score the same packed records, seeded random code and sign words with
+    """The vector-search launches (1M packed keys, d=1024, 4-bit, 1024 query rows, top-10 fused into
+    the search kernel; tq_scores and the fp16-operand tq_search) against the oracle's exact top-10
+    over the whole database, for 8 of the query rows.  Both sides score the same packed records, seeded random code and sign words with
     unit key norms and residual norms of the 3-bit stage's size, so no oracle input comes from the
     GPU; the compression of real inputs is checked on sampled rows above."""
     import torch
@@ -199,16 +209,19 @@ def test_workload5_topk_against_oracle(tq):
     keys = (torch.from_numpy(rec["codes"].view(np.int32)).cuda(), torch.from_numpy(rec["signs"].view(np.int32)).cuda(),
             torch.from_numpy(rec["norm"].view(np.float16)).cuda(),
             torch.from_numpy(rec["rnorm"].view(np.float16)).cuda())
-    _, ti, tv = tq.tq_scores(p, torch.from_numpy(Q.reshape(1, 1, Nq, d)).cuda(), keys, 1, N, want_scores=False,
-                             topk=k)
-    torch.cuda.synchronize()
-    ti, tv = ti.cpu().numpy()[0, 0], tv.cpu().numpy()[0, 0]
+    qd = torch.from_numpy(Q.reshape(1, 1, Nq, d)).cuda()
+    got = {}
+    for fn in (tq.tq_scores, tq.tq_search):
+        _, ti, tv = fn(p, qd, keys, 1, N, want_scores=False, topk=k)
+        torch.cuda.synchronize()
+        got[fn.__name__] = (ti.cpu().numpy()[0, 0], tv.cpu().numpy()[0, 0])
     rows = np.arange(0, Nq, Nq // 8)
     ora = oracle.scores(Q[rows].reshape(1, 1, len(rows), d), R, S, bits, 1, 1, 1, len(rows), N, rec["codes"],
                         rec["signs"], rec["norm"], rec["rnorm"])[0, 0]
     oi, ov = oracle.topk(ora, k)
-    for j, r in enumerate(rows):
-        check_topk(ti[r], tv[r], ora[j], k, f"row {r}")
-        # where no near-tie straddles the k-th place, the sets are equal
-        if ov[j, k - 1] - np.sort(ora[j])[::-1][k] > 2 * (1e-4 + 1e-3 * abs(ov[j, k - 1])):
-            assert set(ti[r].tolist()) == set(oi[j].tolist()), f"row {r}: top-{k} sets differ"
+    for name, (ti, tv) in got.items():
+        for j, r in enumerate(rows):
+            check_topk(ti[r], tv[r], ora[j], k, f"{name} row {r}")
+            # where no near-tie straddles the k-th place, the sets are equal
+            if ov[j, k - 1] - np.sort(ora[j])[::-1][k] > 2 * (1e-4 + 1e-3 * abs(ov[j, k - 1])):
+                assert set(ti[r].tolist()) == set(oi[j].tolist()), f"{name} row {r}: top-{k} sets differ"

@@ -230,6 +230,57 @@ def test_search_scores_and_topk(tq, cfg):
                     np.testing.assert_array_equal(ti[0, 0, r], order)
 
 
+@pytest.mark.parametrize("cfg", [
+    dict(d=1024, m=512, bits=4, Nq=130, T=300),   # the vector-search width
+    dict(d=128, m=64, bits=3, Nq=200, T=1000),    # two row blocks, ragged keys
+    dict(d=128, m=64, bits=3, Nq=16, T=500),      # few rows: not the tensor-core search path
+])
+def test_search_fp16_operands(tq, cfg):
+    """tq_search (single fp16 operand products) on unit keys and queries: every score within the
+    header's bound 2^-10 ||k|| (sum_i |q_rot,i c_i| + rho gamma sum_j |(S q)_j|) of the exact
+    tq_scores; at the vector-search width (d = 1024, typical error ~1e-5) also within the scores
+    tolerance of the oracle, which d = 128 (typical error ~3e-5, tail ~1.5e-4) does not promise;
+    top-k against the oracle.  Shapes outside the tensor-core search run exactly as tq_scores."""
+    import torch
+    c = cfg
+    d, m, bits, Nq, T = c["d"], c["m"], c["bits"], c["Nq"], c["T"]
+    seed = 700 + d + T
+    R = synth.rotation(d, seed)
+    S = synth.gaussian(m, d, seed + 1)
+    K = synth.unit_rows(T, d, seed + 2)
+    k = oracle.compress(K, R, S, bits, is_key=True)
+    q = synth.unit_rows(Nq, d, seed + 3).reshape(1, 1, Nq, d)
+    ora = oracle.scores(q, R, S, bits, 1, 1, 1, Nq, T, k["codes"], k["signs"], k["norm"], k["rnorm"])
+    p = _params(tq, R, S, bits, m)
+    qd = torch.from_numpy(q).cuda()
+    s16, _, _ = tq.tq_search(p, qd, _to_dev(k), 1, T)
+    s32, _, _ = tq.tq_scores(p, qd, _to_dev(k), 1, T)
+    torch.cuda.synchronize()
+    s16, s32 = s16.cpu().numpy()[0, 0].astype(np.float64), s32.cpu().numpy()[0, 0].astype(np.float64)
+    if d >= 1024 or Nq <= 64:
+        check_close(s16, ora[0, 0], "fp16-operand scores")
+    # the stated bound, per score, from the oracle's own quantities
+    nk = np.array([oracle.f16_bits_to_f64(int(h)) for h in as_u16(k["norm"])])
+    rho = np.array([oracle.f16_bits_to_f64(int(h)) for h in as_u16(k["rnorm"])])
+    idx = np.stack([oracle.unpack_codes(w, d, bits - 1) for w in k["codes"]])  # [T, d]
+    cvals = oracle.codebook(d, bits - 1)[1][idx]                     # centroids c[idx] [T, d]
+    qr = q[0, 0].astype(np.float64) @ R.astype(np.float64).T       # q_rot [Nq, d]
+    sq = q[0, 0].astype(np.float64) @ S.astype(np.float64).T       # S q [Nq, m]
+    gamma = math.sqrt(math.pi / 2) / m
+    bound = 2.0 ** -10 * nk[None, :] * (np.abs(qr) @ np.abs(cvals).T + gamma * rho[None, :] *
+                                        np.abs(sq).sum(1)[:, None])
+    err = np.abs(s16 - s32)
+    assert np.all(err <= bound + 1e-6), f"max excess {np.max(err - bound)}"
+    if Nq <= 64:
+        np.testing.assert_array_equal(s16, s32)
+    for k_ in (1, 10):
+        _, ti, tv = tq.tq_search(p, qd, _to_dev(k), 1, T, want_scores=False, topk=k_)
+        torch.cuda.synchronize()
+        ti, tv = ti.cpu().numpy()[0, 0], tv.cpu().numpy()[0, 0]
+        for r in range(0, Nq, 7):
+            check_topk(ti[r], tv[r], ora[0, 0, r], k_, f"k={k_} row {r}")
+
+
 def test_search_topk_exact_ties(tq):
     # identical keys, many query rows: ties resolve to the smaller token index across CTAs too
     import torch
