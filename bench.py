@@ -183,25 +183,50 @@ def run_reference(args):
 
 # -------------------------------------------------------------------- GPU arm
 
-def traffic_per_unit(kernel: str):
-    """DRAM bytes per unit of `kernel` from the committed ncu summary, or None when the kernel's
-    source has changed since the counters were taken (the summary records its sha1)."""
+def source_closure(path: str) -> list[str]:
+    """Repo-relative paths of `path` and of every file it includes with #include "...", followed
+    recursively (looked up beside the including file, then in the package's csrc/ and include/)."""
+    import re
+    seen, todo = [], [path]
+    dirs = [os.path.join("kv_cache_vector_compress_b200", "csrc"), "include"]
+    while todo:
+        rel = todo.pop()
+        if rel in seen:
+            continue
+        seen.append(rel)
+        try:
+            text = open(os.path.join(ROOT, rel)).read()
+        except OSError:
+            continue
+        for inc in re.findall(r'^\s*#\s*include\s+"([^"]+)"', text, flags=re.M):
+            for base in [os.path.dirname(rel)] + dirs:
+                cand = os.path.normpath(os.path.join(base, inc))
+                if os.path.exists(os.path.join(ROOT, cand)):
+                    todo.append(cand)
+                    break
+    return sorted(seen)
+
+
+def sources_sha1(path: str) -> str:
+    """sha1 over the kernel source and everything it includes (names and contents)."""
     import hashlib
+    h = hashlib.sha1()
+    for rel in source_closure(path):
+        h.update(rel.encode() + b"\0")
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()
+
+
+def traffic_per_unit(kernel: str):
+    """DRAM bytes per unit of `kernel` from the committed counters (profiles/dram_traffic.json),
+    or None when the kernel's source or anything it includes has changed since they were taken."""
     try:
-        lines = open(os.path.join(ROOT, "profiles", "dram_traffic.md")).read().splitlines()
-    except OSError:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))["kernels"][kernel]
+    except (OSError, ValueError, KeyError):
         return None
-    for ln in lines:
-        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
-        if len(cells) >= 4 and cells[0] == kernel:
-            src, sha, per_unit = cells[1], cells[2], cells[3]
-            try:
-                cur = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:12]
-                if cur == sha:
-                    return float(per_unit)
-            except (OSError, ValueError):
-                return None
-    return None
+    if sources_sha1(rec["source"]) != rec["sources_sha1"]:
+        return None
+    return float(rec["bytes_per_unit"])
 
 
 def run_tq(args):
@@ -294,7 +319,8 @@ def run_tq(args):
     ms = tqdist.max_over_ranks(ms, device="cuda")
     ms_step = ms / args.steps
 
-    # end to end through the public API: pinned host K/V in, attention output out
+    # end to end through the C-ABI with host buffers: one tq_compress_attend_host call per step
+    # copies the pinned host K/V/Q in, compresses, attends and copies the output back
     hK = torch.empty((n, d), dtype=torch.float16, pin_memory=True)
     hV = torch.empty((n, d), dtype=torch.float16, pin_memory=True)
     hQ = torch.empty((B, Hq, Nq, d), dtype=torch.float32, pin_memory=True)
@@ -302,25 +328,23 @@ def run_tq(args):
     hK.copy_(K)
     hV.copy_(V)
     hQ.copy_(Q)
-    e2e_steps = max(1, min(args.steps, 5))
+    hscr = torch.empty(tq.tq_compress_attend_host_scratch_bytes(p, torch.float16, B, Hq, Hkv, Nq, T),
+                       dtype=torch.uint8, device="cuda")
 
     def e2e_step():
-        K.copy_(hK, non_blocking=True)
-        V.copy_(hV, non_blocking=True)
-        Q.copy_(hQ, non_blocking=True)
-        step()
-        hO.copy_(out, non_blocking=True)
+        tq.tq_compress_attend_host(p, hK, hV, hQ, Hkv, T, keys, vals, hO, scratch=hscr)
 
-    e2e_step()
+    for _ in range(args.warmup):
+        e2e_step()
     barrier()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
     a0.record(stream)
-    for _ in range(e2e_steps):
+    for _ in range(args.steps):
         e2e_step()
     a1.record(stream)
     barrier()
-    e2e_ms = a0.elapsed_time(a1) / e2e_steps
+    e2e_ms = a0.elapsed_time(a1) / args.steps
     e2e_ms = tqdist.max_over_ranks(e2e_ms, device="cuda")
 
     cpu = None

@@ -290,6 +290,34 @@ tq_status tq_attend_merge(const tq_params *p, const float *partials, int parts, 
                           int32_t *dev_status, tq_stream_t stream);
 
 /*
+ * tq_compress_attend_host -- one whole prefill-and-decode step from host memory: copy fp16/fp32
+ * keys, values and queries from the host, compress the keys and values into the caller's device
+ * cache arrays, attend, and copy the attention output back to the host, all enqueued on `stream`
+ * (the cache wrapper's prefill then attention_scores / weighted value sum: "turboquant-pytorch",
+ * nav.superapi.store, 核心 API and 常见使用模式).
+ *   k_host, v_host : host [B, Hkv, T, dim] of dtype (TQ_F16 or TQ_F32)
+ *   q_host         : host fp32 [B, Hq, Nq, dim]
+ *   kcodes .. vnorm: device cache arrays for B * Hkv * T records (tq_compress_keys /
+ *                    tq_compress_values layouts), overwritten
+ *   scale          : as tq_attend
+ *   out_host       : host fp32 [B, Hq, Nq, dim]; valid once `stream` has been synchronised
+ *   scratch        : device buffer of tq_compress_attend_host_scratch_bytes(...) bytes (staging
+ *                    of the inputs and the output, and the attention's scratch)
+ * Host buffers should be page-locked (cudaHostAlloc) for the copies to run asynchronously; with
+ * pageable memory the CUDA runtime stages them and the call returns later.  The host buffers
+ * must stay valid and unmodified until the stream has been synchronised.  Errors: those of
+ * tq_compress_keys, tq_compress_values and tq_attend (host pointers may not be NULL).
+ */
+size_t tq_compress_attend_host_scratch_bytes(const tq_params *p, tq_dtype dtype, int B, int Hq, int Hkv,
+                                             int Nq, int64_t T);
+tq_status tq_compress_attend_host(const tq_params *p, const void *k_host, const void *v_host, tq_dtype dtype,
+                                  const float *q_host, int B, int Hq, int Hkv, int Nq, int64_t T,
+                                  uint32_t *kcodes, uint32_t *ksigns, uint16_t *knorm, uint16_t *krnorm,
+                                  uint32_t *vcodes, uint16_t *vnorm, float scale, float *out_host,
+                                  void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                                  tq_stream_t stream);
+
+/*
  * tq_attend_static -- tq_attend for callers that cannot allocate device memory when they call.
  * (The pages have no counterpart: this is an addition of the library.)
  * A serving loop whose device memory is all handed to its own pool up front, or code that must

@@ -302,6 +302,71 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
     return from_cuda(e);
 }
 
+namespace {
+struct HostStepScratch {
+    size_t k, v, q, o, att, total;
+};
+HostStepScratch host_step_layout(const tq_params *p, tq_dtype dtype, int B, int Hq, int Hkv, int Nq, int64_t T) {
+    HostStepScratch L;
+    const size_t es = dtype == TQ_F16 ? 2 : 4;
+    const size_t kv = (size_t)B * Hkv * (size_t)T * p->dim * es;
+    const size_t qo = (size_t)B * Hq * (size_t)Nq * p->dim * 4;
+    size_t o = 0;
+    L.k = o;
+    o = align_up(o + kv, 256);
+    L.v = o;
+    o = align_up(o + kv, 256);
+    L.q = o;
+    o = align_up(o + qo, 256);
+    L.o = o;
+    o = align_up(o + qo, 256);
+    L.att = o;
+    o += tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, T);
+    L.total = o;
+    return L;
+}
+}  // namespace
+
+size_t tq_compress_attend_host_scratch_bytes(const tq_params *p, tq_dtype dtype, int B, int Hq, int Hkv, int Nq,
+                                             int64_t T) {
+    if (check_params(p, true) != TQ_OK) return 0;
+    if (dtype != TQ_F16 && dtype != TQ_F32) return 0;
+    if (tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, T) == 0) return 0;
+    return host_step_layout(p, dtype, B, Hq, Hkv, Nq, T).total;
+}
+
+tq_status tq_compress_attend_host(const tq_params *p, const void *k_host, const void *v_host, tq_dtype dtype,
+                                  const float *q_host, int B, int Hq, int Hkv, int Nq, int64_t T, uint32_t *kcodes,
+                                  uint32_t *ksigns, uint16_t *knorm, uint16_t *krnorm, uint32_t *vcodes,
+                                  uint16_t *vnorm, float scale, float *out_host, void *scratch, size_t scratch_bytes,
+                                  int32_t *dev_status, tq_stream_t stream) {
+    tq_status st = check_params(p, true);
+    if (st != TQ_OK) return st;
+    if (!k_host || !v_host || !q_host || !out_host) return TQ_ERR_INVALID_ARG;
+    if (dtype != TQ_F16 && dtype != TQ_F32) return TQ_ERR_INVALID_ARG;
+    const size_t need = tq_compress_attend_host_scratch_bytes(p, dtype, B, Hq, Hkv, Nq, T);
+    if (need == 0) return TQ_ERR_INVALID_ARG;
+    if (!scratch || !aligned16(scratch) || scratch_bytes < need) return TQ_ERR_INVALID_ARG;
+    const HostStepScratch L = host_step_layout(p, dtype, B, Hq, Hkv, Nq, T);
+    char *base = (char *)scratch;
+    const int64_t n = (int64_t)B * Hkv * T;
+    const size_t es = dtype == TQ_F16 ? 2 : 4;
+    const size_t kvb = (size_t)n * p->dim * es, qob = (size_t)B * Hq * (size_t)Nq * p->dim * 4;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(base + L.k, k_host, kvb, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + L.v, v_host, kvb, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + L.q, q_host, qob, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    st = tq_compress_keys(p, base + L.k, dtype, n, kcodes, ksigns, knorm, krnorm, dev_status, stream);
+    if (st != TQ_OK) return st;
+    st = tq_compress_values(p, base + L.v, dtype, n, vcodes, vnorm, dev_status, stream);
+    if (st != TQ_OK) return st;
+    st = tq_attend(p, (const float *)(base + L.q), B, Hq, Hkv, Nq, T, kcodes, ksigns, knorm, krnorm, vcodes, vnorm,
+                   scale, (float *)(base + L.o), base + L.att, scratch_bytes - L.att, dev_status, stream);
+    if (st != TQ_OK) return st;
+    return from_cuda(cudaMemcpyAsync(out_host, base + L.o, qob, cudaMemcpyDeviceToHost, s));
+}
+
 tq_status tq_attend_partial(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
                             const uint32_t *kcodes, const uint32_t *ksigns, const uint16_t *knorm,
                             const uint16_t *krnorm, const uint32_t *vcodes, const uint16_t *vnorm, float scale,

@@ -67,6 +67,11 @@ _lib.tq_append_attend.argtypes = [_PP, _P, _P, _P, _I, _I, _I, _I, _I, _I64, _I6
 _lib.tq_append_attend.restype = _I
 _lib.tq_attend_scratch_bytes.argtypes = [_PP, _I, _I, _I, _I, _I64]
 _lib.tq_attend_scratch_bytes.restype = _SZ
+_lib.tq_compress_attend_host_scratch_bytes.argtypes = [_PP, _I, _I, _I, _I, _I, _I64]
+_lib.tq_compress_attend_host_scratch_bytes.restype = _SZ
+_lib.tq_compress_attend_host.argtypes = [_PP, _P, _P, _I, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P,
+                                         ctypes.c_float, _P, _P, _SZ, _P, _P]
+_lib.tq_compress_attend_host.restype = _I
 _lib.tq_attend.argtypes = [_PP, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
                            _SZ, _P, _P]
 _lib.tq_attend.restype = _I
@@ -91,6 +96,7 @@ EXPORTS = ["tq_status_string", "tq_version", "tq_codebook", "tq_codebook_beta", 
            "tq_prepare", "tq_prepare_law",
            "tq_compress_keys", "tq_compress_values", "tq_scores_scratch_bytes", "tq_scores", "tq_search",
            "tq_attend_scratch_bytes", "tq_attend", "tq_attend_partial", "tq_attend_merge", "tq_append_attend",
+           "tq_compress_attend_host_scratch_bytes", "tq_compress_attend_host",
            "tq_selftest_wait_timeout",
            "tq_attend_static"]
 
@@ -261,6 +267,31 @@ def tq_search(p: Params, q: torch.Tensor, keys, Hkv: int, T: int, want_scores: b
 
 def tq_attend_scratch_bytes(p: Params, B, Hq, Hkv, Nq, T) -> int:
     return _lib.tq_attend_scratch_bytes(p.ref, B, Hq, Hkv, Nq, T)
+
+
+def tq_compress_attend_host_scratch_bytes(p: Params, dtype: torch.dtype, B, Hq, Hkv, Nq, T) -> int:
+    return _lib.tq_compress_attend_host_scratch_bytes(p.ref, TQ_F16 if dtype == torch.float16 else TQ_F32, B, Hq,
+                                                      Hkv, Nq, T)
+
+
+def tq_compress_attend_host(p: Params, k_host: torch.Tensor, v_host: torch.Tensor, q_host: torch.Tensor, Hkv: int,
+                            T: int, keys, values, out_host: torch.Tensor, scale: float = 0.0, scratch=None,
+                            dev_status=None):
+    """One step from host memory: k_host / v_host [B, Hkv, T, dim] (fp16 or fp32) and q_host
+    [B, Hq, Nq, dim] fp32 on the host (pinned for asynchronous copies), compressed into the device
+    cache arrays keys (codes, signs, norm, rnorm) and values (codes, norm), attended, and the
+    output written to out_host [B, Hq, Nq, dim] fp32 (valid after the stream synchronises)."""
+    B, Hq, Nq, _ = q_host.shape
+    kc, ks, kn, kr = keys
+    vc, vn = values
+    need = tq_compress_attend_host_scratch_bytes(p, k_host.dtype, B, Hq, Hkv, Nq, T)
+    if scratch is None:
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=kc.device)
+    _check(_lib.tq_compress_attend_host(p.ref, _ptr(k_host), _ptr(v_host), _dtype_code(k_host), _ptr(q_host), B, Hq,
+                                        Hkv, Nq, T, _ptr(kc), _ptr(ks), _ptr(kn), _ptr(kr), _ptr(vc), _ptr(vn),
+                                        float(scale), _ptr(out_host), _ptr(scratch), scratch.numel(),
+                                        _ptr(dev_status), _stream()), "tq_compress_attend_host")
+    return out_host
 
 
 def tq_attend(p: Params, q: torch.Tensor, keys, values, Hkv: int, T: int, scale: float = 0.0, out=None,

@@ -176,6 +176,21 @@ def test_argument_errors_return_before_any_launch(lib):
     assert att(10, out=None) == 1
     assert att(10, sb=16) == 1
     assert att(10, scale=float("nan")) == 1
+    # host-buffer step: missing host pointers, bad dtype, scratch too small
+    L.tq_compress_attend_host.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                          ctypes.c_void_p]
+    host = lambda kh=fake, oh=fake, dt=0, T=10, sb=1 << 40: L.tq_compress_attend_host(
+        P(good), kh, fake, dt, fake, 1, 4, 2, 1, T, fake, fake, fake, fake, fake, fake, 0.0, oh, fake, sb, None,
+        None)
+    assert host(kh=None) == 1
+    assert host(oh=None) == 1
+    assert host(dt=5) == 1
+    assert host(T=0) == 1
+    assert host(sb=16) == 1
     # decode-step append: slot outside the cache, bad dtype, missing or misaligned new rows
     L.tq_append_attend.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,

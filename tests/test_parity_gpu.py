@@ -353,6 +353,53 @@ def test_attend_on_oracle_cache(tq, cfg):
     check_close(out2, ora2, "attend scale=0.02")
 
 
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_compress_attend_host(tq, dtype):
+    """tq_compress_attend_host: host K/V/Q in, host output out, through one C-ABI call.  The cache
+    arrays it writes equal those of tq_compress_keys / tq_compress_values on the same inputs, its
+    output equals tq_attend's over them, and the output matches the oracle's attention over the
+    oracle's own compression of the inputs where the packed records agree (all of them here)."""
+    import torch
+    d, m, bits, B, Hq, Hkv, Nq, T = 128, 64, 3, 2, 8, 2, 1, 300
+    seed = 900 + (dtype == "f32")
+    R = synth.rotation(d, seed)
+    S = synth.gaussian(m, d, seed + 1)
+    n = B * Hkv * T
+    K = synth.gaussian(n, d, seed + 2)
+    V = synth.gaussian(n, d, seed + 3)
+    if dtype == "f16":
+        K, V = K.astype(np.float16), V.astype(np.float16)
+    q = synth.gaussian(B * Hq * Nq, d, seed + 4).reshape(B, Hq, Nq, d)
+    p = _params(tq, R, S, bits, m)
+    hK = torch.from_numpy(K).reshape(B, Hkv, T, d).pin_memory()
+    hV = torch.from_numpy(V).reshape(B, Hkv, T, d).pin_memory()
+    hQ = torch.from_numpy(q).pin_memory()
+    hO = torch.full((B, Hq, Nq, d), float("nan"), dtype=torch.float32).pin_memory()
+    kz = (torch.zeros((n, p.key_words()), dtype=torch.int32, device="cuda"),
+          torch.zeros((n, m // 32), dtype=torch.int32, device="cuda"),
+          torch.zeros(n, dtype=torch.float16, device="cuda"), torch.zeros(n, dtype=torch.float16, device="cuda"))
+    vz = (torch.zeros((n, p.value_words()), dtype=torch.int32, device="cuda"),
+          torch.zeros(n, dtype=torch.float16, device="cuda"))
+    tq.tq_compress_attend_host(p, hK, hV, hQ, Hkv, T, kz, vz, hO)
+    torch.cuda.synchronize()
+    Kd, Vd = hK.cuda().view(n, d), hV.cuda().view(n, d)
+    kt, vt = tq.tq_compress_keys(p, Kd), tq.tq_compress_values(p, Vd)
+    ref = tq.tq_attend(p, hQ.cuda(), kt, vt, Hkv, T)
+    torch.cuda.synchronize()
+    for a, b in zip(kz + vz, kt + vt):
+        assert torch.equal(a, b)
+    np.testing.assert_array_equal(hO.numpy(), ref.cpu().numpy())
+    k = oracle.compress(K.astype(np.float32) if dtype == "f32" else K, R, S, bits, is_key=True)
+    v = oracle.compress(V.astype(np.float32) if dtype == "f32" else V, R, None, bits, is_key=False)
+    ora = oracle.attend(q, R, S, bits, B, Hq, Hkv, Nq, T, k["codes"], k["signs"], k["norm"], k["rnorm"],
+                        v["codes"], v["norm"])
+    same = ((as_u32(kz[0]) == k["codes"]).all(1) & (as_u32(kz[1]) == k["signs"]).all(1)
+            & (as_u16(kz[2]) == k["norm"]) & (as_u16(kz[3]) == k["rnorm"])
+            & (as_u32(vz[0]) == v["codes"]).all(1) & (as_u16(vz[1]) == v["norm"]))
+    if same.all():
+        check_close(hO, ora, "host-step attend")
+
+
 def test_end_to_end_workload1(tq):
     """Compress with the GPU, attend with the GPU; oracle does the same from the same inputs."""
     import torch
