@@ -226,8 +226,10 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
  * ("turboquant-pytorch", nav.superapi.store, 核心 API: TurboQuantKVCache with append_key,
  * append_value, attention_scores; "TurboQuant: онлайн-квантование векторов без калибровки",
  * ai-manual.ru, "Где TurboQuant выстреливает, а где нет?": keys and values compressed during
- * generation).  The compression runs inside the attention kernel, in the CTA whose context range
- * holds slot t, so the step launches no separate compress kernel (tensor-core attention shapes).
+ * generation).  With at most 4 query rows per KV head (the bit-plane attention shapes) the new
+ * rows go through the tensor-core compress kernels into a staging part of the scratch and are
+ * scattered to slot t; with 5 to 64 rows (register-MMA attention shapes) the compression runs
+ * inside the attention kernel, in the CTA whose context range holds slot t.
  *   q            : device fp32 [B, Hq, Nq, dim]
  *   k_new, v_new : device [B, Hkv, dim] of dtype (TQ_F16 or TQ_F32), 16-byte aligned
  *   t            : the slot the new token takes, 0 <= t < t_cap; slots 0 .. t-1 hold the cache
@@ -236,8 +238,8 @@ tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
  *                  tq_compress_keys / tq_compress_values; slot t is overwritten
  *   scale, out   : as tq_attend; the attention covers slots 0 .. t (t + 1 tokens)
  *   scratch      : tq_attend_scratch_bytes(p, B, Hq, Hkv, Nq, t + 1) bytes
- * For shapes outside the tensor-core attention kernel (dim 64, 128 or 256 with proj_dim = dim / 2
- * and 2-4 bit keys) the append is a small kernel of its own, launched before the attention.
+ * For other shapes (outside dim 64, 128 or 256 with proj_dim = dim / 2 and 2-4 bit keys) the
+ * append is a small kernel of its own, launched before the attention.
  * Returns the errors of tq_attend.
  */
 tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new, const void *v_new,

@@ -261,8 +261,9 @@ size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int N
     ScoreProblem sp = make_problem(B, Hq, Hkv, Nq, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                    nullptr);
     const AttendPlan plan = plan_attend(P, sp);
+    // bit-plane path: query operands, then the staging of tq_append_attend's new records
     return qprep_bytes(P, sp) + attend_partials_bytes(P, sp, plan.splits) +
-           (plan.planes ? planes_frag_bytes(P, sp) : 0);
+           (plan.planes ? planes_frag_bytes(P, sp) + append_stage_bytes(P, sp) : 0);
 }
 
 tq_status tq_attend(const tq_params *p, const float *q, int B, int Hq, int Hkv, int Nq, int64_t T,
@@ -423,7 +424,6 @@ tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new
                            uint32_t *kcodes, uint32_t *ksigns, uint16_t *knorm, uint16_t *krnorm,
                            uint32_t *vcodes, uint16_t *vnorm, float scale, float *out, void *scratch,
                            size_t scratch_bytes, int32_t *dev_status, tq_stream_t stream) {
-    (void)dev_status;
     tq_status st = check_params(p, true);
     if (st != TQ_OK) return st;
     if (t < 0 || t_cap < 1 || t >= t_cap) return TQ_ERR_INVALID_ARG;
@@ -458,8 +458,9 @@ tq_status tq_append_attend(const tq_params *p, const float *q, const void *k_new
     uint32_t *frag = (uint32_t *)((char *)partials + attend_partials_bytes(P, sp, plan.splits));
     cudaError_t e = plan.planes ? cudaSuccess : launch_qprep(P, sp, qprep, s);
     if (plan.planes) {
-        // the append kernel, then the bit-plane attention over slots 0..t of the strided cache
-        if (e == cudaSuccess) e = launch_append(P, sp, s);
+        // the new rows through the compress kernels into a staging area, scattered to slot t; then
+        // the bit-plane attention over slots 0..t of the strided cache
+        if (e == cudaSuccess) e = launch_append_staged(P, sp, (char *)frag + planes_frag_bytes(P, sp), dev_status, s);
         ScoreProblem rd = sp;
         rd.knew = rd.vnew = nullptr;
         if (e == cudaSuccess) e = launch_planes(P, rd, scale, frag, plan.pp, true, out, partials, s);

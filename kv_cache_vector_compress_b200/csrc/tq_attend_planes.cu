@@ -4,7 +4,7 @@
 // Math (asymmetric scores from the compressed keys, softmax, weighted sum over the MSE-
 // dequantized values; "turboquant-pytorch", nav.superapi.store, 常见使用模式 and 核心 API):
 //   s_tr = ||k_t|| ( <q_rot_r, c[kidx_t]> + rho_t sqrt(pi/2)/m <sq_r, 2 sign_t - 1> )
-//   o_rot_r = sum_t softmax_t(scale s_tr) ||v_t|| c[vidx_t],   out_r = R^T o_rot_r (combine kernel)
+//   o_rot_r = sum_t softmax_t(scale s_tr) ||v_t|| c[vidx_t],   out_r = R^T o_rot_r
 //
 // Walsh form of the codebook.  The Lloyd-Max codebooks are exactly antisymmetric
 // (c[K-1-k] = -c[k]), so as a function of the code bits b_0..b_{beta-1} (s_i = 2 b_i - 1)
@@ -24,8 +24,11 @@
 //     the softmax weights times the value norms are rounded to 16-bit fixed point relative to the
 //     largest value norm of the CTA's token range (absolute error 2^-17 of it per token).
 // Two passes per CTA over a range of at most kPRange tokens: (1) scores of the whole range into
-// shared memory (and the row maxima); (2) the fixed-point weights, then the value products.  The
-// per-range (max, sum, o_rot) partials are merged by attend_combine_kernel.
+// shared memory (and the row maxima); (2) the fixed-point weights, then the value products.  Each
+// CTA writes its range's (max, sum, o_rot) partial; the last CTA of a (batch, KV head) slice to
+// finish (an atomic count per slice) merges them by log-sum-exp and applies R^T, or writes the
+// merged partial for tq_attend_partial.  A separate kernel (planes_qfrag_kernel) prepares each
+// slice's query operands first.
 #include <math.h>
 
 #include "tq_common.cuh"

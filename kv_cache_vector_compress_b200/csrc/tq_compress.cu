@@ -68,6 +68,57 @@ cudaError_t launch_append_npl(const Prepared &P, const ScoreProblem &sp, cudaStr
     return cudaGetLastError();
 }
 
+// Records i of the staging arrays (the new rows, compressed contiguously) to record i * Ts + tnew
+// of the caches: one thread per word of a record, the norms by the record's first thread.
+__global__ void scatter_new_kernel(ScoreProblem sp, int kw, int sw, int vw, const uint32_t *__restrict__ skc,
+                                   const uint32_t *__restrict__ sks, const uint32_t *__restrict__ svc,
+                                   const uint16_t *__restrict__ skn, const uint16_t *__restrict__ skr,
+                                   const uint16_t *__restrict__ svn) {
+    const int64_t nsl = (int64_t)sp.B * sp.Hkv;
+    const int per = kw + sw + vw;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < nsl * per;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / per;
+        const int w = (int)(e % per);
+        const int64_t rec = i * sp.Ts + sp.tnew;
+        if (w < kw) {
+            sp.kcodes_w[rec * kw + w] = skc[i * kw + w];
+        } else if (w < kw + sw) {
+            sp.ksigns_w[rec * sw + (w - kw)] = sks[i * sw + (w - kw)];
+        } else {
+            sp.vcodes_w[rec * vw + (w - kw - sw)] = svc[i * vw + (w - kw - sw)];
+        }
+        if (w == 0) {
+            sp.knorm_w[rec] = skn[i];
+            sp.krnorm_w[rec] = skr[i];
+            sp.vnorm_w[rec] = svn[i];
+        }
+    }
+}
+
+struct AppendStage {
+    size_t kc, ks, vc, kn, kr, vn, total;
+};
+AppendStage append_stage_layout(const Prepared &P, const ScoreProblem &sp) {
+    const size_t nsl = (size_t)sp.B * sp.Hkv;
+    AppendStage L;
+    size_t o = 0;
+    L.kc = o;
+    o = align_up(o + nsl * P.kbeta * (P.d / 32) * 4, 256);
+    L.ks = o;
+    o = align_up(o + nsl * (P.m / 32) * 4, 256);
+    L.vc = o;
+    o = align_up(o + nsl * P.vbeta * (P.d / 32) * 4, 256);
+    L.kn = o;
+    o = align_up(o + nsl * 2, 256);
+    L.kr = o;
+    o = align_up(o + nsl * 2, 256);
+    L.vn = o;
+    o = align_up(o + nsl * 2, 256);
+    L.total = o;
+    return L;
+}
+
 template <int NPL>
 cudaError_t launch_npl(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,
                        uint32_t *codes, uint32_t *signs, uint16_t *norm, uint16_t *rnorm,
@@ -100,6 +151,25 @@ cudaError_t launch_append(const Prepared &P, const ScoreProblem &sp, cudaStream_
         case 1024: return launch_append_npl<32>(P, sp, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+size_t append_stage_bytes(const Prepared &P, const ScoreProblem &sp) { return append_stage_layout(P, sp).total; }
+
+cudaError_t launch_append_staged(const Prepared &P, const ScoreProblem &sp, void *stage, int32_t *dev_status,
+                                 cudaStream_t s) {
+    const AppendStage L = append_stage_layout(P, sp);
+    char *b = (char *)stage;
+    uint32_t *skc = (uint32_t *)(b + L.kc), *sks = (uint32_t *)(b + L.ks), *svc = (uint32_t *)(b + L.vc);
+    uint16_t *skn = (uint16_t *)(b + L.kn), *skr = (uint16_t *)(b + L.kr), *svn = (uint16_t *)(b + L.vn);
+    const int64_t nsl = (int64_t)sp.B * sp.Hkv;
+    cudaError_t e = launch_compress(P, true, sp.knew, sp.new_f16, nsl, skc, sks, skn, skr, dev_status, s);
+    if (e == cudaSuccess) e = launch_compress(P, false, sp.vnew, sp.new_f16, nsl, svc, nullptr, svn, nullptr, dev_status, s);
+    if (e != cudaSuccess) return e;
+    const int kw = P.kbeta * (P.d / 32), sw = P.m / 32, vw = P.vbeta * (P.d / 32);
+    const int64_t work = nsl * (kw + sw + vw);
+    const unsigned blocks = (unsigned)((work + 255) / 256 < 148 * 8 ? (work + 255) / 256 : 148 * 8);
+    scatter_new_kernel<<<blocks, 256, 0, s>>>(sp, kw, sw, vw, skc, sks, svc, skn, skr, svn);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_compress(const Prepared &P, bool is_key, const void *x, bool x_f16, int64_t n,

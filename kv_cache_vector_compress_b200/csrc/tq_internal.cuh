@@ -159,6 +159,11 @@ struct ScoreProblem {
 
 // Compress the new key / value of every slice into record s * Ts + tnew (sp.knew, sp.vnew set).
 cudaError_t launch_append(const Prepared &P, const ScoreProblem &sp, cudaStream_t s);
+// The same append through the compress kernels: the new rows are compressed contiguously into
+// `stage` (append_stage_bytes), then scattered to record s * Ts + tnew.
+size_t append_stage_bytes(const Prepared &P, const ScoreProblem &sp);
+cudaError_t launch_append_staged(const Prepared &P, const ScoreProblem &sp, void *stage, int32_t *dev_status,
+                                 cudaStream_t s);
 size_t qprep_bytes(const Prepared &P, const ScoreProblem &sp);
 int attend_splits(const ScoreProblem &sp);
 size_t attend_partials_bytes(const Prepared &P, const ScoreProblem &sp, int splits);

@@ -382,14 +382,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
                 rb = sp.krnorm[rec];
             }
         };
-        uint2 cu[KB], nu[KB];
-        uint32_t crb = 0, nrb = 0;
-        bool cval = false, nval = false;
-        if (grp < total) fetch(grp, cu, crb, cval);
-        for (int gk = grp; gk < total; gk += kDecGroups) {
-            if (gk + kDecGroups < total) fetch(gk + kDecGroups, nu, nrb, nval);
+        // decode K-block step gk from its fetched words into its TMEM stage; false on abort
+        auto decode = [&](int gk, const uint2 (&cu)[KB], uint32_t crb, bool cval) -> bool {
             const int st = gk % kSStages, kbi = gk % NKB;
-            if (gk >= kSStages && !mbar_wait(&bars[kSEmpty + st], ((gk / kSStages) - 1) & 1, abort_s)) break;
+            if (gk >= kSStages && !mbar_wait(&bars[kSEmpty + st], ((gk / kSStages) - 1) & 1, abort_s))
+                return false;
             tc_fence_after();
             const uint32_t ta = tq + st * kAStageCols;
             if (kbi < DKB) {
@@ -455,10 +452,27 @@ __global__ void __launch_bounds__(kSThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kAFull + st]);
-#pragma unroll
-            for (int p = 0; p < KB; ++p) cu[p] = nu[p];
-            crb = nrb;
-            cval = nval;
+            return true;
+        };
+        // three word buffers in turn: each step's words are fetched two of this group's steps
+        // ahead, so their loads have two decodes to land in
+        constexpr int D1 = kDecGroups, D2 = 2 * kDecGroups;
+        uint2 b0[KB], b1[KB], b2[KB];
+        uint32_t r0 = 0, r1 = 0, r2 = 0;
+        bool v0 = false, v1 = false, v2 = false;
+        if (grp < total) fetch(grp, b0, r0, v0);
+        if (grp + D1 < total) fetch(grp + D1, b1, r1, v1);
+        for (int gk = grp; gk < total; gk += 3 * D1) {
+            if (gk + D2 < total) fetch(gk + D2, b2, r2, v2);
+            if (!decode(gk, b0, r0, v0)) break;
+            const int g1 = gk + D1;
+            if (g1 >= total) break;
+            if (g1 + D2 < total) fetch(g1 + D2, b0, r0, v0);
+            if (!decode(g1, b1, r1, v1)) break;
+            const int g2 = g1 + D1;
+            if (g2 >= total) break;
+            if (g2 + D2 < total) fetch(g2 + D2, b1, r1, v1);
+            if (!decode(g2, b2, r2, v2)) break;
         }
     } else {
         // -------------------------------------------------------- scores and top-k
