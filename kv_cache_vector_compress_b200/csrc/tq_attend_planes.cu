@@ -177,13 +177,23 @@ __device__ __forceinline__ int32_t digit(int64_t &q) {
 // registers with one funnel shift and two masks.  The B value is Q / e with
 // Q = round(gamma / Lambda), gamma = 2 alpha_S q_rot[32 g + beta] (code planes) or 2 sq[...]
 // (signs), and Lambda = max |gamma| / 2^30 per row and kind.
+// Rows of R^T and S^T staged in shared memory per chunk of input coordinates (at most ~96 KB).
+template <int D>
+struct QfragChunk {
+    static constexpr int NQ = D + D / 2;
+    static constexpr int KC = (NQ * D * 4 <= 96 * 1024) ? D : (96 * 1024) / (NQ * 4) / 32 * 32;
+    static constexpr uint32_t BYTES = (uint32_t)KC * NQ * 4;
+};
+
 template <int D, int KB>
 __global__ void __launch_bounds__(256) planes_qfrag_kernel(Prepared P, ScoreProblem sp, float scale,
                                                          uint32_t *__restrict__ frag) {
     using C = PlanesCfg<D, KB, 1>;
     constexpr int NQ = D + C::M;
     constexpr int NTH = 256;
-    __shared__ float qraw[kPRows][D];
+    static_assert(QfragChunk<D>::NQ == NQ && D % QfragChunk<D>::KC == 0, "chunking");
+    extern __shared__ __align__(16) float wsm[];  // [KC][NQ] rows of R^T | S^T
+    __shared__ __align__(16) float4 qT[D];        // qT[j] = (q_0[j], q_1[j], q_2[j], q_3[j])
     __shared__ float qs[kPRows][NQ];
     __shared__ uint32_t Qd[kPRows][C::NK][32];  // the four balanced base-256 digits, as bytes
     __shared__ double alpha[8];
@@ -195,7 +205,7 @@ __global__ void __launch_bounds__(256) planes_qfrag_kernel(Prepared P, ScoreProb
     const int b = (int)(sl / sp.Hkv), kv = (int)(sl % sp.Hkv);
     const int G = sp.Hq / sp.Hkv, nrows = G * sp.Nq;
     uint32_t *out = frag + sl * (int64_t)C::SLW;
-    // the slice's query rows (zero beyond nrows)
+    // the slice's query rows (zero beyond nrows), coordinate-major
     for (int e = tid; e < kPRows * D; e += NTH) {
         const int r = e / D, c = e % D;
         float v = 0.f;
@@ -203,7 +213,7 @@ __global__ void __launch_bounds__(256) planes_qfrag_kernel(Prepared P, ScoreProb
             const int g = r / sp.Nq, i = r % sp.Nq;
             v = sp.q[(((int64_t)b * sp.Hq + (int64_t)kv * G + g) * sp.Nq + i) * D + c];
         }
-        qraw[r][c] = v;
+        (&qT[c].x)[r] = v;
     }
     if (tid < C::KPL) {
         const int sub = walsh_subset(KB, tid), K = 1 << KB;
@@ -218,32 +228,48 @@ __global__ void __launch_bounds__(256) planes_qfrag_kernel(Prepared P, ScoreProb
     }
     if (tid < kPRows * 2 * 4) (&esum[0][0][0])[tid] = 0;
     __syncthreads();
-    // q_rot = R q and S q: four outputs per warp at a time, the lanes split each dot product
-    // (all of a step's weight loads are issued before the first product)
-    constexpr int OPW = 4;
-    for (int c0 = warp * OPW; c0 < NQ; c0 += (NTH / 32) * OPW) {
-        float wv[OPW][D / 32];
+    // q_rot = R q and S q: thread t takes outputs t, t + 256, ...; the rows of R^T and S^T (input
+    // coordinate j: the weights of all outputs) come through shared memory in chunks of KC
+    // coordinates, copied with every load of a chunk in flight at once
+    constexpr int KC = QfragChunk<D>::KC;
+    constexpr int OPT = (NQ + NTH - 1) / NTH;
+    float acc[OPT][kPRows];
 #pragma unroll
-        for (int o = 0; o < OPW; ++o) {
-            const int c = min(c0 + o, NQ - 1);
-            const float *wrow = c < D ? P.R + (int64_t)c * D : P.S + (int64_t)(c - D) * D;
+    for (int o = 0; o < OPT; ++o)
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i) wv[o][i] = wrow[lane + 32 * i];
+        for (int r = 0; r < kPRows; ++r) acc[o][r] = 0.f;
+    for (int k0 = 0; k0 < D; k0 += KC) {
+        if (k0 > 0) __syncthreads();  // the previous chunk is consumed
+        for (int e = tid; e < KC * (NQ / 4); e += NTH) {
+            const int j = e / (NQ / 4), c4 = 4 * (e % (NQ / 4));
+            const float *src = c4 < D ? P.RT + (int64_t)(k0 + j) * D + c4 : P.ST + (int64_t)(k0 + j) * C::M + (c4 - D);
+            cp_async<16>(wsm + j * NQ + c4, src);
         }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+#pragma unroll 4
+        for (int j = 0; j < KC; ++j) {
+            const float4 q4 = qT[k0 + j];
 #pragma unroll
-        for (int o = 0; o < OPW; ++o) {
-            float acc[kPRows] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < D / 32; ++i)
-#pragma unroll
-                for (int r = 0; r < kPRows; ++r) acc[r] = fmaf(wv[o][i], qraw[r][lane + 32 * i], acc[r]);
-#pragma unroll
-            for (int r = 0; r < kPRows; ++r) {
-                float v = acc[r];
-                for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(kFull, v, sh);
-                if (lane == 0 && c0 + o < NQ) qs[r][c0 + o] = v;
+            for (int o = 0; o < OPT; ++o) {
+                const int c = tid + o * NTH;
+                if (c < NQ) {
+                    const float w = wsm[j * NQ + c];
+                    acc[o][0] = fmaf(w, q4.x, acc[o][0]);
+                    acc[o][1] = fmaf(w, q4.y, acc[o][1]);
+                    acc[o][2] = fmaf(w, q4.z, acc[o][2]);
+                    acc[o][3] = fmaf(w, q4.w, acc[o][3]);
+                }
             }
         }
+    }
+#pragma unroll
+    for (int o = 0; o < OPT; ++o) {
+        const int c = tid + o * NTH;
+        if (c < NQ)
+#pragma unroll
+            for (int r = 0; r < kPRows; ++r) qs[r][c] = acc[o][r];
     }
     __syncthreads();
     // gamma of (row, product, position k): 2 alpha_S q_rot[32 g + bit] or 2 (S q)[32 g' + bit]
@@ -906,8 +932,11 @@ cudaError_t launch_planes_t(const Prepared &P, const ScoreProblem &sp, float sca
                             int range, int splits, float *out, float *partials, cudaStream_t s, int mp) {
     using C = PlanesCfg<D, KB, VB>;
     const int64_t slices = (int64_t)sp.B * sp.Hkv;
-    planes_qfrag_kernel<D, KB><<<(unsigned)slices, 256, 0, s>>>(P, sp, ATTEND ? scale : 1.0f, frag);
-    cudaError_t e = cudaGetLastError();
+    auto qk = planes_qfrag_kernel<D, KB>;
+    cudaError_t e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QfragChunk<D>::BYTES);
+    if (e != cudaSuccess) return e;
+    qk<<<(unsigned)slices, 256, QfragChunk<D>::BYTES, s>>>(P, sp, ATTEND ? scale : 1.0f, frag);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const PlanesSmem L = planes_smem<D, KB, VB, ATTEND>(range, splits);
     auto kern = planes_attend_kernel<D, KB, VB, ATTEND>;
