@@ -281,6 +281,40 @@ def test_search_fp16_operands(tq, cfg):
             check_topk(ti[r], tv[r], ora[0, 0, r], k_, f"k={k_} row {r}")
 
 
+@pytest.mark.parametrize("fn", ["tq_scores", "tq_search"])
+def test_sharded_search_topk_merge(tq, fn):
+    """The sharded vector search on one GPU: a database split into two row ranges, the fused
+    top-k of each range (indices made global by the range's offset) merged by dist.merge_topk,
+    equals the top-k of one call over the whole database, and matches the oracle's top-k."""
+    import torch
+    from kv_cache_vector_compress_b200 import dist
+    d, m, bits, Nq, T, k = 1024, 512, 4, 130, 700, 10
+    R = synth.rotation(d, 41)
+    S = synth.gaussian(m, d, 42)
+    K = synth.unit_rows(T, d, 43)
+    kk = oracle.compress(K, R, S, bits, is_key=True)
+    q = synth.unit_rows(Nq, d, 44).reshape(1, 1, Nq, d)
+    ora = oracle.scores(q, R, S, bits, 1, 1, 1, Nq, T, kk["codes"], kk["signs"], kk["norm"], kk["rnorm"])
+    p = _params(tq, R, S, bits, m)
+    qd = torch.from_numpy(q).cuda()
+    call = getattr(tq, fn)
+    dev = _to_dev(kk)
+    _, ti, tv = call(p, qd, dev, 1, T, want_scores=False, topk=k)
+    cut = 300  # a range boundary inside a 128-key tile
+    parts_v, parts_i = [], []
+    for a, b in ((0, cut), (cut, T)):
+        sub = tuple(x[a:b].clone() for x in dev)  # each shard in its own (16-byte aligned) buffers
+        _, si, sv = call(p, qd, sub, 1, b - a, want_scores=False, topk=k)
+        parts_v.append(sv)
+        parts_i.append(si.to(torch.int64) + a)
+    mi, mv = dist.merge_topk(torch.cat(parts_v, -1), torch.cat(parts_i, -1), k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(mi.cpu().numpy(), ti.cpu().numpy().astype(np.int64))
+    np.testing.assert_array_equal(mv.cpu().numpy(), tv.cpu().numpy())
+    for r in range(0, Nq, 13):
+        check_topk(ti[0, 0, r].cpu().numpy(), tv[0, 0, r].cpu().numpy(), ora[0, 0, r], k, f"{fn} row {r}")
+
+
 def test_search_topk_exact_ties(tq):
     # identical keys, many query rows: ties resolve to the smaller token index across CTAs too
     import torch
