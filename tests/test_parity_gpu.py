@@ -468,6 +468,8 @@ def test_end_to_end_workload1(tq):
     dict(d=128, m=64, bits=2, B=1, Hkv=1, G=16, Nq=1, t=333, cap=400, f16=True),    # two row groups
     dict(d=32, m=32, bits=3, B=2, Hkv=1, G=2, Nq=1, t=50, cap=64, f16=True),        # append kernel + CUDA-core attention
     dict(d=128, m=128, bits=3, B=1, Hkv=2, G=2, Nq=3, t=200, cap=256, f16=False),   # proj_dim = dim: same path
+    dict(d=128, m=64, bits=3, B=1, Hkv=2, G=2, Nq=2, t=77, cap=90, f16=False),      # bit-plane shape, fp32 rows
+    dict(d=256, m=128, bits=2, B=1, Hkv=2, G=4, Nq=1, t=600, cap=700, f16=True),    # bit-plane shape, wide head
 ])
 def test_append_attend(tq, cfg):
     """tq_append_attend writes the oracle's records for the new token into slot t, leaves every other
