@@ -458,16 +458,38 @@ __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
     }
     const float lam_c = __uint_as_float(crow[8]), lam_s = __uint_as_float(crow[9]);
 
-    // ---- value norms of the range (and their maximum)
+    // ---- value norms of the range (and their maximum), every load of a thread in flight at once;
+    // the Walsh coefficients of the value codebook (read at the end of the CTA)
+    __shared__ double va_s[8];
     float nmax = 0.f;
     if constexpr (ATTEND) {
-        for (int i = tid; i < len; i += NT) {
-            const uint16_t h = sp.vnorm[rec_base + i];
-            vnb[i] = h;
-            nmax = fmaxf(nmax, f16_bits_to_f32(h));
+        constexpr int NPT = (kPRange + NT - 1) / NT;
+        uint16_t hv[NPT];
+#pragma unroll
+        for (int k = 0; k < NPT; ++k) {
+            const int i = tid + k * NT;
+            hv[k] = i < len ? sp.vnorm[rec_base + i] : (uint16_t)0;
+        }
+#pragma unroll
+        for (int k = 0; k < NPT; ++k) {
+            const int i = tid + k * NT;
+            if (i < len) {
+                vnb[i] = hv[k];
+                nmax = fmaxf(nmax, f16_bits_to_f32(hv[k]));
+            }
         }
         nmax = warp_max(nmax);
         if (lane == 0) red[64 + warp] = nmax;
+        if (tid < C::VPL) {
+            constexpr int K = 1 << VB;
+            const int sub = walsh_subset(VB, tid);
+            double a = 0.0;
+            for (int idx = 0; idx < K; ++idx) {
+                const int par = __popc(idx & sub) ^ __popc(sub);  // number of zero bits in S, mod 2
+                a += (par & 1) ? -(double)P.cb->vc[idx] : (double)P.cb->vc[idx];
+            }
+            va_s[tid] = a / K;
+        }
     }
     if constexpr (!C::KREG) __syncthreads();
 
@@ -806,21 +828,10 @@ __global__ void __launch_bounds__(PlanesCfg<D, KB, VB>::NW * 32)
                     for (int e = 0; e < 4; ++e) cv[s][t][e] += src[((s * C::TPW + t) * 4 + e) * 32];
         }
     }
-    // Walsh coefficients of the value codebook
+    // Walsh coefficients of the value codebook (computed in the prologue; barriers since)
     double va[C::VPL];
-    {
-        constexpr int K = 1 << VB;
 #pragma unroll
-        for (int s = 0; s < C::VPL; ++s) {
-            const int sub = walsh_subset(VB, s);
-            double a = 0.0;
-            for (int idx = 0; idx < K; ++idx) {
-                const int par = __popc(idx & sub) ^ __popc(sub);  // number of zero bits in S, mod 2
-                a += (par & 1) ? -(double)P.cb->vc[idx] : (double)P.cb->vc[idx];
-            }
-            va[s] = a / K;
-        }
-    }
+    for (int s = 0; s < C::VPL; ++s) va[s] = va_s[s];
     // row t4: sum of weights and of fixed-point weights over the range
     float lrow = 0.f;
     int64_t utot = 0;
