@@ -273,7 +273,7 @@ def test_search_fp16_operands(tq, cfg):
     assert np.all(err <= bound + 1e-6), f"max excess {np.max(err - bound)}"
     if Nq <= 64:
         np.testing.assert_array_equal(s16, s32)
-    for k_ in (1, 10):
+    for k_ in (1, 10, 20):  # 20: past the fused top-k, a separate pass over the fp16-operand scores
         _, ti, tv = tq.tq_search(p, qd, _to_dev(k), 1, T, want_scores=False, topk=k_)
         torch.cuda.synchronize()
         ti, tv = ti.cpu().numpy()[0, 0], tv.cpu().numpy()[0, 0]
