@@ -31,63 +31,74 @@ inline int rows_per_pass(int d, int m, int cap_regs) {
 
 // ------------------------------------------------------------------ query prep
 
-constexpr int kQpR = 64;   // query rows per block tile
-constexpr int kQpC = 64;   // output coordinates per block tile
-constexpr int kQpK = 16;   // input coordinates per shared-memory step
+constexpr int kQpR = 64;    // query rows per block tile
+constexpr int kQpC = 128;   // output coordinates per block tile
+constexpr int kQpK = 16;    // input coordinates per shared-memory step
 
 // q_rot = R q and sq = S q as one fp32 GEMM, out[r][i] = sum_j q[r][j] W[j][i] with
-// W = [R^T | S^T]: 64 x 64 output tiles, 4 x 4 per thread, operands staged in shared memory.
-// Every output is accumulated by fmaf in ascending j, so the result does not depend on the
-// tiling.
+// W = [R^T | S^T]: 64 x 128 output tiles, 4 x 8 per thread (columns tx * 4 and 64 + tx * 4), the
+// next step's operands loaded into registers while the current step computes.  Every output is
+// accumulated by fmaf in ascending j, so the result does not depend on the tiling.
 __global__ void __launch_bounds__(256) qprep_kernel(Prepared P, const float *__restrict__ q, int64_t rows,
                                                     float *__restrict__ out) {
-    __shared__ float qs[kQpK][kQpR + 4];  // q tile, transposed
+    __shared__ __align__(16) float qs[kQpK][kQpR + 4];  // q tile, transposed
     __shared__ __align__(16) float ws[kQpK][kQpC];
     const int d = P.d, m = P.m, n = d + m;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int c0 = blockIdx.x * kQpC;
+    // this thread's loads of a step: one float4 of q (row lr, k 4 lk4..) and two of W (k lw, columns
+    // lc and lc + 64)
+    const int lr = tid >> 2, lk4 = 4 * (tid & 3), lw = tid >> 4, lc = 4 * (tid & 15);
+    auto wload = [&](int j, int c) -> float4 {
+        const int i = c0 + c;
+        if (i < d) return *(const float4 *)(P.RT + (int64_t)j * d + i);
+        if (i < n) return *(const float4 *)(P.ST + (int64_t)j * m + (i - d));
+        return make_float4(0.f, 0.f, 0.f, 0.f);
+    };
     for (int64_t r0 = (int64_t)blockIdx.y * kQpR; r0 < rows; r0 += (int64_t)gridDim.y * kQpR) {
-        float acc[4][4];
+        float acc[4][8];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+            for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+        const bool qok = r0 + lr < rows;
+        float4 gq = qok ? *(const float4 *)(q + (r0 + lr) * d + lk4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 gw0 = wload(lw, lc), gw1 = wload(lw, lc + 64);
         for (int k0 = 0; k0 < d; k0 += kQpK) {
-            for (int e = tid; e < kQpR * kQpK; e += 256) {
-                const int r = e / kQpK, k = e % kQpK;
-                qs[k][r] = r0 + r < rows ? q[(r0 + r) * d + k0 + k] : 0.f;
-            }
-            for (int e = tid; e < kQpK * kQpC; e += 256) {
-                const int k = e / kQpC, c = e % kQpC, i = c0 + c, j = k0 + k;
-                float w = 0.f;
-                if (i < d) w = P.RT[(int64_t)j * d + i];
-                else if (i < n) w = P.ST[(int64_t)j * m + (i - d)];
-                ws[k][c] = w;
-            }
+            __syncthreads();  // the previous step's tiles are consumed
+            qs[lk4 + 0][lr] = gq.x;
+            qs[lk4 + 1][lr] = gq.y;
+            qs[lk4 + 2][lr] = gq.z;
+            qs[lk4 + 3][lr] = gq.w;
+            *(float4 *)&ws[lw][lc] = gw0;
+            *(float4 *)&ws[lw][lc + 64] = gw1;
             __syncthreads();
+            if (k0 + kQpK < d) {
+                const int k1 = k0 + kQpK;
+                gq = qok ? *(const float4 *)(q + (r0 + lr) * d + k1 + lk4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                gw0 = wload(k1 + lw, lc);
+                gw1 = wload(k1 + lw, lc + 64);
+            }
 #pragma unroll
             for (int k = 0; k < kQpK; ++k) {
-                float a[4];
+                const float4 a4 = *(const float4 *)&qs[k][ty * 4];
+                const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float4 b0 = *(const float4 *)&ws[k][tx * 4];
+                const float4 b1 = *(const float4 *)&ws[k][64 + tx * 4];
+                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-                for (int t = 0; t < 4; ++t) a[t] = qs[k][ty * 4 + t];
-                const float4 b = *(const float4 *)&ws[k][tx * 4];
+                for (int t = 0; t < 4; ++t)
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    acc[t][0] = fmaf(b.x, a[t], acc[t][0]);
-                    acc[t][1] = fmaf(b.y, a[t], acc[t][1]);
-                    acc[t][2] = fmaf(b.z, a[t], acc[t][2]);
-                    acc[t][3] = fmaf(b.w, a[t], acc[t][3]);
-                }
+                    for (int u = 0; u < 8; ++u) acc[t][u] = fmaf(b[u], a[t], acc[t][u]);
             }
-            __syncthreads();
         }
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const int64_t r = r0 + ty * 4 + t;
             if (r >= rows) continue;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = c0 + tx * 4 + u;
+            for (int u = 0; u < 8; ++u) {
+                const int i = c0 + (u < 4 ? tx * 4 + u : 64 + tx * 4 + (u - 4));
                 if (i < n) out[r * n + i] = acc[t][u];
             }
         }
