@@ -365,6 +365,10 @@ def test_search_topk_increasing_scores(tq):
     dict(d=256, m=128, bits=2, B=1, Hkv=1, G=4, Nq=1, T=3000),
     dict(d=256, m=128, bits=4, B=1, Hkv=1, G=4, Nq=1, T=513),
     dict(d=32, m=32, bits=1 + 1, B=1, Hkv=1, G=1, Nq=1, T=127),
+    # bit-plane shapes (at most 4 query rows per KV head, proj_dim = dim / 2) at their edges
+    dict(d=64, m=32, bits=3, B=2, Hkv=1, G=4, Nq=1, T=1),      # a single token
+    dict(d=128, m=64, bits=4, B=1, Hkv=2, G=2, Nq=2, T=31),    # under one 32-token stage
+    dict(d=64, m=32, bits=2, B=1, Hkv=1, G=1, Nq=3, T=2049),   # three ranges, 3 rows, ragged tail
 ])
 def test_attend_on_oracle_cache(tq, cfg):
     import torch
