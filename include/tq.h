@@ -208,7 +208,8 @@ tq_status tq_search(const tq_params *p, const float *q, int B, int Hq, int Hkv, 
  *   keys   : as tq_scores;  vcodes / vnorm: the arrays of tq_compress_values
  *   scale  : softmax temperature; <= 0 selects 1/sqrt(dim)
  *   out    : device fp32 [B, Hq, Nq, dim]
- *   scratch: device buffer of tq_attend_scratch_bytes(...) bytes (split-context partials)
+ *   scratch: device buffer of tq_attend_scratch_bytes(...) bytes (query operands, split-context
+ *            partials, and room to stage the new records of tq_append_attend)
  * T must be >= 1.
  */
 size_t tq_attend_scratch_bytes(const tq_params *p, int B, int Hq, int Hkv, int Nq, int64_t T);
