@@ -18,6 +18,10 @@
 // Warp roles: 0 streams the B tiles and owns TMEM, 1 issues the MMAs, 2..9 convert the A
 // tiles (two groups taking alternate K-blocks), 10..13 run the epilogue.  Two TMEM slots of
 // 256 columns keep one chunk's epilogue under the next chunk's MMAs.
+// fp16 values with d <= 256 (one rotation chunk) take the input itself as the A operand: fp16 is
+// exact, so ACC = x (R 2^8)(hi + lo) needs two products per k-step, the converters only copy
+// the rows into the swizzled stage, and the epilogue takes ||x|| = ||ACC|| / 2^8 from the
+// accumulator (R orthogonal, to the 2^-22 of its split) before coding y = ACC / ||ACC||.
 #include "tq_common.cuh"
 #include "tq_internal.cuh"
 #include "tq_sm100.cuh"
@@ -183,6 +187,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int KWPT = BETA * (d / 32);
     const int SWPT = G.m / 32;
     const int NC = G.nchunks();
+    const bool exact = !IS_KEY && F16 && G.nr == 1;  // A = the fp16 input itself (see the header)
     const int64_t ntiles = (n + kBRows - 1) / kBRows;
     const int my_tiles = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
 
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             const uint32_t o = 32 * k;
                             mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kb | k) ? 1u : 0u);
                             mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
-                            mma_ss(acc, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
+                            if (!exact) mma_ss(acc, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
                         }
                         mma_commit(&bars[kBEmpty + st]);
                     }
@@ -309,9 +314,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
         for (int i = 0; ok && i < my_tiles; ++i) {
             const int64_t v = (blockIdx.x + (int64_t)i * gridDim.x) * kBRows + r;
             const bool valid = v < n;
-            // ||x|| in fp32 from the input row
+            // ||x|| in fp32 from the input row (the exact path takes it from the accumulator)
             float ss = 0.f;
-            if (valid) {
+            if (valid && !exact) {
                 if (F16) {
                     const uint4 *xr = (const uint4 *)((const __half *)xin + v * d);
                     for (int j = 0; j < d / 8; ++j) {
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
             }
             const float nrm = sqrtf(ss);
             const float us = nrm > 0.f ? (float)(1 << kUScaleLog2) / nrm : 0.f;
-            if (valid && cg == 0) norm[v] = f32_to_f16_bits(nrm);
+            if (valid && cg == 0 && !exact) norm[v] = f32_to_f16_bits(nrm);
             bool have_codes = false;
             for (int c = 0; ok && c < NC; ++c) {
                 const int nkb = G.nkb(c);
@@ -361,6 +366,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             ok = false;
                             break;
                         }
+                        if (F16 && exact) {
+                            // the fp16 row itself, one 16-byte chunk of 8 coordinates at a time
+#pragma unroll
+                            for (int cc = 0; cc < 8; ++cc)
+                                *(uint4 *)(ah + rowb + (((uint32_t)cc ^ (r & 7)) << 4)) = q[cc];
+                        } else {
 #pragma unroll
                         for (int cc = 0; cc < 8; ++cc) {
                             float f[8];
@@ -388,6 +399,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             const uint32_t off = rowb + (((uint32_t)cc ^ (r & 7)) << 4);
                             *(uint4 *)(ah + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
                             *(uint4 *)(al + off) = make_uint4(lv4[0], lv4[1], lv4[2], lv4[3]);
+                        }
                         }
                     } else {
                         // correction: -c[idx] 2^14 for coordinates 64 kbc .. 64 kbc + 63 from the
@@ -467,6 +479,25 @@ __global__ void __launch_bounds__(kBThreads, 1)
                 tc_fence_after();
                 const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16) + slot * kBChunk;
                 const int ng = G.width(c) / 32, g0 = G.n0(c) / 32;
+                // exact path: ACC = 2^8 R x; ||x|| = ||ACC|| / 2^8 and y = ACC / ||ACC||
+                float yscale = kYUnscale;
+                if (exact) {
+                    float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll 1
+                    for (int g = 0; g < ng; ++g) {
+                        uint32_t a[32];
+                        tmem_ld32(tl + 32 * g, a);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const float2 a2 = make_float2(__uint_as_float(a[2 * k]), __uint_as_float(a[2 * k + 1]));
+                            ss2 = __ffma2_rn(a2, a2, ss2);
+                        }
+                    }
+                    const float na = sqrtf(ss2.x + ss2.y);
+                    yscale = na > 0.f ? 1.0f / na : 0.f;
+                    if (valid) norm[v] = f32_to_f16_bits(na * (1.0f / (float)(1 << kRScaleLog2)));
+                }
                 if (c < G.nr) {
                     // codes of rotated coordinates 32 (g0 + g) .. + 31, planar words
 #pragma unroll 1
@@ -479,7 +510,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         for (int p = 0; p < BETA; ++p) wp[p] = 0u;
 #pragma unroll
                         for (int l = 0; l < 32; ++l) {
-                            const float y = __uint_as_float(a[l]) * kYUnscale;
+                            const float y = __uint_as_float(a[l]) * yscale;
                             const uint32_t idx = big_bucket<BETA>(y, bnd_r);
 #pragma unroll
                             for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
