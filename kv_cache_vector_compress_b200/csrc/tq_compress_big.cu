@@ -18,10 +18,13 @@
 // Warp roles: 0 streams the B tiles and owns TMEM, 1 issues the MMAs, 2..9 convert the A
 // tiles (two groups taking alternate K-blocks), 10..13 run the epilogue.  Two TMEM slots of
 // 256 columns keep one chunk's epilogue under the next chunk's MMAs.
-// fp16 values with d <= 256 (one rotation chunk) take the input itself as the A operand: fp16 is
-// exact, so ACC = x (R 2^8)(hi + lo) needs two products per k-step, the converters only copy
-// the rows into the swizzled stage, and the epilogue takes ||x|| = ||ACC|| / 2^8 from the
-// accumulator (R orthogonal, to the 2^-22 of its split) before coding y = ACC / ||ACC||.
+// fp16 input with d <= 256 (one rotation chunk; keys also m <= 128) takes the input itself as the
+// A operand: fp16 is exact, so x (R 2^8)(hi + lo) needs two products per k-step, the converters
+// only copy the rows into the swizzled stage, and the epilogue takes ||x|| = ||ACC|| / 2^8 from
+// the rotation accumulator (R orthogonal, to the 2^-22 of its split) before coding
+// y = ACC / ||ACC||.  Keys accumulate x (S 2^8)^T = ||ACC|| S u and the correction
+// -2^18 S' c[idx] side by side in the projection slot; the epilogue forms
+// 2^18 p = ACC_S 2^18 / ||ACC|| + ACC_c before taking its sign.
 #include "tq_common.cuh"
 #include "tq_internal.cuh"
 #include "tq_sm100.cuh"
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int KWPT = BETA * (d / 32);
     const int SWPT = G.m / 32;
     const int NC = G.nchunks();
-    const bool exact = !IS_KEY && F16 && G.nr == 1;  // A = the fp16 input itself (see the header)
+    const bool exact = F16 && G.nr == 1 && (!IS_KEY || G.m <= 128);  // A = the fp16 input (see the header)
     const int64_t ntiles = (n + kBRows - 1) / kBRows;
     const int my_tiles = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
 
@@ -280,10 +283,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t acc = tmem + slot * kBChunk;
+                    const uint32_t acc0 = tmem + slot * kBChunk;
                     const uint32_t idesc = idesc_f16_f32(kBRows, G.width(c));
                     const int nkb = G.nkb(c);
                     for (int kb = 0; kb < nkb; ++kb, ++gk) {
+                        // exact keys: the correction K-blocks go to their own accumulator
+                        const bool corr = kb >= dkb;
+                        const uint32_t acc = (exact && corr) ? acc0 + 128 : acc0;
+                        const int kb0 = (exact && corr) ? kb - dkb : kb;  // first K-block of acc: 0
                         const int st = gk % kBStages;
                         if (!mbar_wait(&bars[kBFull + st], (gk / kBStages) & 1, abort_s)) {
                             ok = false;
@@ -295,9 +302,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint32_t o = 32 * k;
-                            mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kb | k) ? 1u : 0u);
+                            mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kb0 | k) ? 1u : 0u);
                             mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
-                            if (!exact) mma_ss(acc, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
+                            if (!exact || corr) mma_ss(acc, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
                         }
                         mma_commit(&bars[kBEmpty + st]);
                     }
@@ -470,6 +477,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
             const int64_t v = (blockIdx.x + (int64_t)i * gridDim.x) * kBRows + r;
             const bool valid = v < n;
             float ee = 0.f;
+            float na = 0.f;  // exact path: ||ACC|| of the rotation chunk (2^8 ||x||)
             for (int c = 0; c < NC; ++c, ++gc) {
                 const int slot = gc & 1;
                 if (!mbar_wait(&bars[kBAccFull + slot], (gc >> 1) & 1, abort_s)) {
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                 const int ng = G.width(c) / 32, g0 = G.n0(c) / 32;
                 // exact path: ACC = 2^8 R x; ||x|| = ||ACC|| / 2^8 and y = ACC / ||ACC||
                 float yscale = kYUnscale;
-                if (exact) {
+                if (exact && c < G.nr) {
                     float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll 1
                     for (int g = 0; g < ng; ++g) {
@@ -494,7 +502,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             ss2 = __ffma2_rn(a2, a2, ss2);
                         }
                     }
-                    const float na = sqrtf(ss2.x + ss2.y);
+                    na = sqrtf(ss2.x + ss2.y);
                     yscale = na > 0.f ? 1.0f / na : 0.f;
                     if (valid) norm[v] = f32_to_f16_bits(na * (1.0f / (float)(1 << kRScaleLog2)));
                 }
@@ -539,11 +547,25 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     // d (a few 1e-5 of p at d = 1024), so projections with |p| < kSignRecheck are
                     // recomputed in double by the warp, from x, the codes, S and S'.
                     const int64_t vbase = v - lane;
+                    // exact path: 2^18 p = ACC_S 2^18 / ||ACC|| + ACC_c (columns 128 on)
+                    const float pscale = na > 0.f ? (float)(1 << (kUScaleLog2 + kRScaleLog2)) / na : 0.f;
 #pragma unroll 1
                     for (int g = 0; g < ng; ++g) {
                         uint32_t a[32];
                         tmem_ld32(tl + 32 * g, a);
                         tmem_ld_wait();
+                        if (exact) {
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                uint32_t b16[16];
+                                tmem_ld16(tl + 128 + 32 * g + 16 * hh, b16);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int l = 0; l < 16; ++l)
+                                    a[16 * hh + l] = __float_as_uint(
+                                        fmaf(__uint_as_float(a[16 * hh + l]), pscale, __uint_as_float(b16[l])));
+                            }
+                        }
                         uint32_t sw = 0, unc = 0;
 #pragma unroll
                         for (int l = 0; l < 32; ++l) {
