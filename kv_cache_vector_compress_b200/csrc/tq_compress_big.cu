@@ -113,6 +113,19 @@ __device__ __forceinline__ uint32_t big_bucket(float y, const float (&b)[16]) {
     }
 }
 
+// The same search with the boundaries read from shared memory (b_s[0..2^BETA-2]) by index, for
+// 3 and 4 bits, where the register form needs 3 and 11 selects per coordinate.
+template <int BETA>
+__device__ __forceinline__ uint32_t big_bucket_s(float y, const float *b_s) {
+    uint32_t idx = 0;
+#pragma unroll
+    for (int p = BETA - 1; p >= 0; --p) {
+        const uint32_t t = y > b_s[idx + (1u << p) - 1];
+        idx += t << p;
+    }
+    return idx;
+}
+
 __device__ __forceinline__ uint32_t hsplit2(float a, float b, bool lo) {
     const __half ha = __float2half_rn(a), hb = __float2half_rn(b);
     if (!lo) return (uint32_t)__half_as_ushort(ha) | ((uint32_t)__half_as_ushort(hb) << 16);
@@ -519,13 +532,20 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
                         for (int l = 0; l < 32; ++l) {
                             const float y = __uint_as_float(a[l]) * yscale;
-                            const uint32_t idx = big_bucket<BETA>(y, bnd_r);
+                            const uint32_t idx = BETA >= 3 ? big_bucket_s<BETA>(y, bnd_s) : big_bucket<BETA>(y, bnd_r);
 #pragma unroll
                             for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
                             if (IS_KEY) {
-                                float cv = cen_r[0];
+                                // 3 MSE bits: one shared-memory read (the 8 centroids in 8 banks)
+                                // instead of a chain of 7 selects; fewer bits keep the selects
+                                float cv;
+                                if constexpr (BETA >= 3) {
+                                    cv = cen_s[idx];
+                                } else {
+                                    cv = cen_r[0];
 #pragma unroll
-                                for (int k = 1; k < (1 << BETA); ++k) cv = idx == (uint32_t)k ? cen_r[k] : cv;
+                                    for (int k = 1; k < (1 << BETA); ++k) cv = idx == (uint32_t)k ? cen_r[k] : cv;
+                                }
                                 const float e = y - cv;
                                 ee = fmaf(e, e, ee);
                             }
