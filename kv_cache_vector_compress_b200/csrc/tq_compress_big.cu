@@ -47,10 +47,10 @@ constexpr uint32_t kBStage = 2 * kATile + 2 * kBTileMax;  // A hi, A lo, B hi, B
 constexpr int kUScaleLog2 = 10;               // U = u 2^10
 constexpr int kCorrScaleLog2 = kUScaleLog2 + kRScaleLog2 - kSScaleLog2;  // correction A scale
 
-enum BBar { kBFull = 0, kBEmpty = 2, kBAccFull = 4, kBAccEmpty = 6, kBCodes = 8 };
+enum BBar { kBFull = 0, kBEmpty = 2, kBAccFull = 4, kBAccEmpty = 6, kBCodes = 8, kBNorm = 10, kBEe = 12 };
 
 struct BigSmem {
-    uint32_t stage, ctab, bnd, cen, bars, misc, total;
+    uint32_t stage, ctab, bnd, cen, bars, misc, xchg, total;
 };
 
 __host__ __device__ inline BigSmem big_smem_layout() {
@@ -68,6 +68,8 @@ __host__ __device__ inline BigSmem big_smem_layout() {
     o += 32 * 8;
     L.misc = o;
     o += 64;
+    L.xchg = o;  // exact path: partial squared norms [2][2][128], partial residual norms [2][128]
+    o += 3 * 2 * 128 * 4;
     L.total = o;
     return L;
 }
@@ -183,7 +185,7 @@ __device__ __noinline__ double exact_projection(const Prepared &P, const BigGeom
     return (nx > 0.0 ? su / nx : 0.0) - sc;
 }
 
-template <bool IS_KEY, int BETA, bool F16>
+template <bool IS_KEY, int BETA, bool F16, bool EX, bool SPLIT>
 __global__ void __launch_bounds__(kBThreads, 1)
     compress_big_kernel(Prepared P, BigGeom G, const void *__restrict__ xin, int64_t n, uint32_t *__restrict__ codes,
                         uint32_t *__restrict__ signs, uint16_t *__restrict__ norm, uint16_t *__restrict__ rnorm,
@@ -203,7 +205,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int KWPT = BETA * (d / 32);
     const int SWPT = G.m / 32;
     const int NC = G.nchunks();
-    const bool exact = F16 && G.nr == 1 && (!IS_KEY || G.m <= 128);  // A = the fp16 input (see the header)
+    // EX: A = the fp16 input itself (see the header).  SPLIT (exact path with a heavier code step):
+    // one converter group (warps 2..5) takes every K-block and eight epilogue warps (6..13, two
+    // column halves) code each tile.
+    constexpr bool exact = EX;
+    constexpr int kEpi0 = SPLIT ? 6 : kBEpiWarp0;
+    constexpr int kNEpi = SPLIT ? 8 : 4;
+    float *xn_s = (float *)(sm + L.xchg);         // [tile parity][half][row] partial ||ACC||^2
+    float *xe_s = xn_s + 2 * 2 * kBRows;          // [tile parity][row] half 1's part of ||y - c||^2
     const int64_t ntiles = (n + kBRows - 1) / kBRows;
     const int my_tiles = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
 
@@ -214,9 +223,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[kBAccFull + s], 1);
-            mbar_init(&bars[kBAccEmpty + s], 4);
+            mbar_init(&bars[kBAccEmpty + s], kNEpi);
         }
-        for (int s = 0; s < 2; ++s) mbar_init(&bars[kBCodes + s], 4);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kBCodes + s], kNEpi);
+            mbar_init(&bars[kBNorm + s], kNEpi);
+            mbar_init(&bars[kBEe + s], 4);
+        }
         *abort_s = 0;
         fence_mbar_init();
     }
@@ -324,9 +337,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     if (ok) mma_commit(&bars[kBAccFull + slot]);
                 }
         }
-    } else if (warp < kBEpiWarp0) {
+    } else if (warp < kEpi0) {
         // -------------------------------------------------------- A tiles, one vector per thread
-        const int cg = (warp - kCvtWarp0) >> 2;           // group: K-block steps gk with gk % 2 == cg
+        const int cg = SPLIT ? 0 : (warp - kCvtWarp0) >> 2;  // group: K-block steps gk with gk % 2 == cg
         const int r = (threadIdx.x - kCvtWarp0 * 32) & 127;  // the vector this thread converts
         const uint32_t rowb = (uint32_t)r * 128;
         int gk = 0;
@@ -367,7 +380,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
             for (int c = 0; ok && c < NC; ++c) {
                 const int nkb = G.nkb(c);
                 for (int kb = 0; kb < nkb; ++kb, ++gk) {
-                    if ((gk & 1) != cg) continue;
+                    if (!SPLIT && (gk & 1) != cg) continue;
                     const int st = gk % kBStages;
                     uint8_t *ah = sm + L.stage + st * kBStage;
                     uint8_t *al = ah + kATile;
@@ -477,6 +490,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         // -------------------------------------------------------- epilogue, one vector per thread
         const int q4 = warp & 3;  // TMEM lane quarter this warp may read
         const int r = 32 * q4 + lane;
+        const int hf = SPLIT ? (warp - kEpi0) >> 2 : 0;  // column half of this warp
+        constexpr int NHF = SPLIT ? 2 : 1;
         float bnd_r[16], cen_r[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -500,12 +515,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
                 tc_fence_after();
                 const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16) + slot * kBChunk;
                 const int ng = G.width(c) / 32, g0 = G.n0(c) / 32;
+                const int gA = hf * ng / NHF, gB = (hf + 1) * ng / NHF;  // this warp's column groups
                 // exact path: ACC = 2^8 R x; ||x|| = ||ACC|| / 2^8 and y = ACC / ||ACC||
                 float yscale = kYUnscale;
                 if (exact && c < G.nr) {
                     float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll 1
-                    for (int g = 0; g < ng; ++g) {
+                    for (int g = gA; g < gB; ++g) {
                         uint32_t a[32];
                         tmem_ld32(tl + 32 * g, a);
                         tmem_ld_wait();
@@ -515,14 +531,28 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             ss2 = __ffma2_rn(a2, a2, ss2);
                         }
                     }
-                    na = sqrtf(ss2.x + ss2.y);
+                    if constexpr (SPLIT) {
+                        // the halves meet in shared memory (slots of tile parity; a slot is next
+                        // written two tiles on, after both halves have released this tile's chunks)
+                        float *xn = xn_s + (i & 1) * 2 * kBRows;
+                        xn[hf * kBRows + r] = ss2.x + ss2.y;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[kBNorm + (i & 1)]);
+                        if (!mbar_wait(&bars[kBNorm + (i & 1)], (i >> 1) & 1, abort_s)) {
+                            ok = false;
+                            break;
+                        }
+                        na = sqrtf(xn[r] + xn[kBRows + r]);
+                    } else {
+                        na = sqrtf(ss2.x + ss2.y);
+                    }
                     yscale = na > 0.f ? 1.0f / na : 0.f;
-                    if (valid) norm[v] = f32_to_f16_bits(na * (1.0f / (float)(1 << kRScaleLog2)));
+                    if (valid && hf == 0) norm[v] = f32_to_f16_bits(na * (1.0f / (float)(1 << kRScaleLog2)));
                 }
                 if (c < G.nr) {
                     // codes of rotated coordinates 32 (g0 + g) .. + 31, planar words
 #pragma unroll 1
-                    for (int g = 0; g < ng; ++g) {
+                    for (int g = gA; g < gB; ++g) {
                         uint32_t a[32];
                         tmem_ld32(tl + 32 * g, a);
                         tmem_ld_wait();
@@ -556,8 +586,22 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         }
                     }
                     if (IS_KEY && c == G.nr - 1) {
-                        // every code word of this tile is out: release the correction operands
-                        if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
+                        // every code word of this tile is out: release the correction operands.
+                        // Exact path: half 1 hands its part of ||y - c||^2 to half 0 first.
+                        if (SPLIT && hf == 1) {
+                            xe_s[(i & 1) * kBRows + r] = ee;
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&bars[kBEe + (i & 1)]);
+                        } else {
+                            if (SPLIT) {
+                                if (!mbar_wait(&bars[kBEe + (i & 1)], (i >> 1) & 1, abort_s)) {
+                                    ok = false;
+                                    break;
+                                }
+                                ee += xe_s[(i & 1) * kBRows + r];
+                            }
+                            if (valid) rnorm[v] = f32_to_f16_bits(sqrtf(ee));
+                        }
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bars[kBCodes + (i & 1)]);
                     }
@@ -570,7 +614,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     // exact path: 2^18 p = ACC_S 2^18 / ||ACC|| + ACC_c (columns 128 on)
                     const float pscale = na > 0.f ? (float)(1 << (kUScaleLog2 + kRScaleLog2)) / na : 0.f;
 #pragma unroll 1
-                    for (int g = 0; g < ng; ++g) {
+                    for (int g = gA; g < gB; ++g) {
                         uint32_t a[32];
                         tmem_ld32(tl + 32 * g, a);
                         tmem_ld_wait();
@@ -631,7 +675,13 @@ cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64
                        uint16_t *norm, uint16_t *rnorm, int32_t *dev_status, cudaStream_t s) {
     const BigSmem L = big_smem_layout();
     const size_t smem = L.total + 1024;
-    auto kern = compress_big_kernel<IS_KEY, BETA, F16>;
+    // the exact path for fp16 input with one rotation chunk; its code step split over eight warps
+    // where it is heavy (keys; values of 3 or 4 bits)
+    const bool ex = F16 && G.nr == 1 && (!IS_KEY || (G.m <= 128 && G.m % 64 == 0));
+    const bool split = ex && (IS_KEY || BETA >= 3);
+    auto kern = split ? compress_big_kernel<IS_KEY, BETA, F16, F16, F16>
+                      : ex ? compress_big_kernel<IS_KEY, BETA, F16, F16, false>
+                           : compress_big_kernel<IS_KEY, BETA, F16, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
