@@ -562,14 +562,17 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
                         for (int l = 0; l < 32; ++l) {
                             const float y = __uint_as_float(a[l]) * yscale;
-                            const uint32_t idx = BETA >= 3 ? big_bucket_s<BETA>(y, bnd_s) : big_bucket<BETA>(y, bnd_r);
+                            // shared-memory tables on the split exact path; elsewhere shared memory
+                            // is busy with both MMA operands, and the register selects are faster
+                            const uint32_t idx =
+                                (SPLIT && BETA >= 3) ? big_bucket_s<BETA>(y, bnd_s) : big_bucket<BETA>(y, bnd_r);
 #pragma unroll
                             for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
                             if (IS_KEY) {
-                                // 3 MSE bits: one shared-memory read (the 8 centroids in 8 banks)
-                                // instead of a chain of 7 selects; fewer bits keep the selects
+                                // split exact path, 3 MSE bits: one shared-memory read (the 8
+                                // centroids in 8 banks) instead of a chain of 7 selects
                                 float cv;
-                                if constexpr (BETA >= 3) {
+                                if constexpr (SPLIT && BETA >= 3) {
                                     cv = cen_s[idx];
                                 } else {
                                     cv = cen_r[0];
