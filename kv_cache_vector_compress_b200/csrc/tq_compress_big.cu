@@ -18,13 +18,14 @@
 // Warp roles: 0 streams the B tiles and owns TMEM, 1 issues the MMAs, 2..9 convert the A
 // tiles (two groups taking alternate K-blocks), 10..13 run the epilogue.  Two TMEM slots of
 // 256 columns keep one chunk's epilogue under the next chunk's MMAs.
-// fp16 input with d <= 256 (one rotation chunk; keys also m <= 128) takes the input itself as the
+// fp16 input with d <= 256 (one rotation chunk; keys also m <= 256) takes the input itself as the
 // A operand: fp16 is exact, so x (R 2^8)(hi + lo) needs two products per k-step, the converters
 // only copy the rows into the swizzled stage, and the epilogue takes ||x|| = ||ACC|| / 2^8 from
 // the rotation accumulator (R orthogonal, to the 2^-22 of its split) before coding
-// y = ACC / ||ACC||.  Keys accumulate x (S 2^8)^T = ||ACC|| S u and the correction
-// -2^18 S' c[idx] side by side in the projection slot; the epilogue forms
-// 2^18 p = ACC_S 2^18 / ||ACC|| + ACC_c before taking its sign.
+// y = ACC / ||ACC||.  Keys then project the residual: p = S u - S' c[idx] = S' (y - c[idx])
+// (S u = S R^T y), so the epilogue writes 2^14 e = 2^14 (y - c[idx]) as fp16 hi | lo back into
+// the rotation slot and the projection chunk multiplies that TMEM operand by (S' 2^4)(hi + lo),
+// three products per k-step into one accumulator; the converters build no correction blocks.
 #include "tq_common.cuh"
 #include "tq_internal.cuh"
 #include "tq_sm100.cuh"
@@ -76,7 +77,7 @@ __host__ __device__ inline BigSmem big_smem_layout() {
 
 // The chunk sequence of one tile: R chunks (rotation outputs), then, for keys, S chunks
 // (projection outputs), each with its K-blocks: d/64 over U, plus d/64 correction blocks for
-// S chunks.
+// S chunks (the residual form of the exact path has only the d/64 blocks of S').
 struct BigGeom {
     int d, m, nr, ns;  // dims; number of R chunks and S chunks
     __host__ __device__ int nchunks() const { return nr + ns; }
@@ -137,6 +138,7 @@ __device__ __forceinline__ uint32_t hsplit2(float a, float b, bool lo) {
 
 constexpr float kSignRecheck = 1e-4f;  // |p| below which a sign is recomputed exactly
 constexpr float kPUnscaleInv = (float)(1 << (kUScaleLog2 + kRScaleLog2));  // ACC = p 2^18
+constexpr float kEScale = (float)(1 << kCorrScaleLog2);  // residual operand 2^14 e
 
 // p_a = S_a . u - S'_a . c[idx] of vector v in double, one warp: lane l takes coordinates
 // 4 l + 128 i .. + 3 (row-major S and S', coalesced); the codes are the ones this CTA has just
@@ -209,6 +211,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
     // one converter group (warps 2..5) takes every K-block and eight epilogue warps (6..13, two
     // column halves) code each tile.
     constexpr bool exact = EX;
+    // RP (exact keys): the projection is p = S' e of the residual e = y - c[idx], which the
+    // epilogue writes back into the rotation slot (fp16 hi | lo of 2^14 e) as the A operand of the
+    // projection chunk, whose B is S' 2^4 (d/64 K-blocks, three products): no converter work
+    constexpr bool RP = EX && IS_KEY;
+    auto nkb_of = [&](int c) { return (RP && c >= G.nr) ? G.d / 64 : G.nkb(c); };
     constexpr int kEpi0 = SPLIT ? 6 : kBEpiWarp0;
     constexpr int kNEpi = SPLIT ? 8 : 4;
     float *xn_s = (float *)(sm + L.xchg);         // [tile parity][half][row] partial ||ACC||^2
@@ -265,22 +272,24 @@ __global__ void __launch_bounds__(kBThreads, 1)
             bool ok = true;
             for (int i = 0; ok && i < my_tiles; ++i)
                 for (int c = 0; ok && c < NC; ++c) {
-                    const int w = G.width(c), n0 = G.n0(c), nkb = G.nkb(c);
+                    const int w = G.width(c), n0 = G.n0(c), nkb = nkb_of(c);
                     const uint32_t bytes = (uint32_t)w * 128;
                     for (int kb = 0; kb < nkb; ++kb, ++gk) {
                         const int st = gk % kBStages;
+                        const bool sp_blk = RP ? c >= G.nr : kb >= dkb;  // a K-block of S'
+                        const int kbs = RP ? kb : kb - dkb;
                         if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
                             ok = false;
                             break;
                         }
                         const uint8_t *src;
                         size_t lo;
-                        if (kb < dkb) {
+                        if (!sp_blk) {
                             const int row0 = c < G.nr ? n0 : d + n0;
                             src = W + ((size_t)kb * wrows + row0) * 128;
                             lo = wlo;
                         } else {
-                            src = Sp + ((size_t)(kb - dkb) * G.m + n0) * 128;
+                            src = Sp + ((size_t)kbs * G.m + n0) * 128;
                             lo = slo;
                         }
                         uint8_t *dst = sm + L.stage + st * kBStage + 2 * kATile;
@@ -304,19 +313,54 @@ __global__ void __launch_bounds__(kBThreads, 1)
             for (int i = 0; ok && i < my_tiles; ++i)
                 for (int c = 0; ok && c < NC; ++c, ++gc) {
                     const int slot = gc & 1;
-                    if (gc >= 2 && !mbar_wait(&bars[kBAccEmpty + slot], ((gc >> 1) - 1) & 1, abort_s)) {
+                    if constexpr (RP) {
+                        // slot 0: rotation of tile i, then its residual; slot 1: its projection
+                        bool w = true;
+                        if (c < G.nr) {
+                            // the projection of tile i - 1 has read the residual in slot 0
+                            if (i >= 1) w = mbar_wait(&bars[kBAccFull + 1], (i - 1) & 1, abort_s);
+                        } else {
+                            // tile i's residual is written; tile i - 1's projection has been read
+                            w = mbar_wait(&bars[kBAccEmpty + 0], i & 1, abort_s);
+                            if (w && i >= 1) w = mbar_wait(&bars[kBAccEmpty + 1], (i - 1) & 1, abort_s);
+                        }
+                        if (!w) {
+                            ok = false;
+                            break;
+                        }
+                    } else if (gc >= 2 && !mbar_wait(&bars[kBAccEmpty + slot], ((gc >> 1) - 1) & 1, abort_s)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t acc0 = tmem + slot * kBChunk;
                     const uint32_t idesc = idesc_f16_f32(kBRows, G.width(c));
-                    const int nkb = G.nkb(c);
+                    const int nkb = nkb_of(c);
+                    if (RP && c >= G.nr) {
+                        // projection: A = 2^14 e (hi | lo per 32 coordinates) in slot 0
+                        for (int kb = 0; kb < nkb; ++kb, ++gk) {
+                            const int st = gk % kBStages;
+                            if (!mbar_wait(&bars[kBFull + st], (gk / kBStages) & 1, abort_s)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t b_hi = sbase + st * kBStage + 2 * kATile, b_lo = b_hi + kBTileMax;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int K = 4 * kb + k;
+                                const uint32_t a_hi = tmem + 32 * (K >> 1) + 8 * (K & 1), a_lo = a_hi + 16;
+                                const uint64_t dh = sdesc_sw128(b_hi + 32 * k), dl = sdesc_sw128(b_lo + 32 * k);
+                                mma_ts(acc0, a_hi, dh, idesc, (kb | k) ? 1u : 0u);
+                                mma_ts(acc0, a_hi, dl, idesc, 1u);
+                                mma_ts(acc0, a_lo, dh, idesc, 1u);
+                            }
+                            mma_commit(&bars[kBEmpty + st]);
+                        }
+                        if (ok) mma_commit(&bars[kBAccFull + slot]);
+                        continue;
+                    }
                     for (int kb = 0; kb < nkb; ++kb, ++gk) {
-                        // exact keys: the correction K-blocks go to their own accumulator
-                        const bool corr = kb >= dkb;
-                        const uint32_t acc = (exact && corr) ? acc0 + 128 : acc0;
-                        const int kb0 = (exact && corr) ? kb - dkb : kb;  // first K-block of acc: 0
                         const int st = gk % kBStages;
                         if (!mbar_wait(&bars[kBFull + st], (gk / kBStages) & 1, abort_s)) {
                             ok = false;
@@ -328,9 +372,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint32_t o = 32 * k;
-                            mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kb0 | k) ? 1u : 0u);
-                            mma_ss(acc, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
-                            if (!exact || corr) mma_ss(acc, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
+                            mma_ss(acc0, sdesc_sw128(a_hi + o), sdesc_sw128(b_hi + o), idesc, (kb | k) ? 1u : 0u);
+                            mma_ss(acc0, sdesc_sw128(a_hi + o), sdesc_sw128(b_lo + o), idesc, 1u);
+                            if (!exact) mma_ss(acc0, sdesc_sw128(a_lo + o), sdesc_sw128(b_hi + o), idesc, 1u);
                         }
                         mma_commit(&bars[kBEmpty + st]);
                     }
@@ -378,13 +422,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
             if (valid && cg == 0 && !exact) norm[v] = f32_to_f16_bits(nrm);
             bool have_codes = false;
             for (int c = 0; ok && c < NC; ++c) {
-                const int nkb = G.nkb(c);
+                const int nkb = nkb_of(c);
                 for (int kb = 0; kb < nkb; ++kb, ++gk) {
                     if (!SPLIT && (gk & 1) != cg) continue;
                     const int st = gk % kBStages;
                     uint8_t *ah = sm + L.stage + st * kBStage;
                     uint8_t *al = ah + kATile;
-                    if (kb < dkb) {
+                    if (RP && c >= G.nr) {
+                        // the projection's A operand is in TMEM: only keep the stage's arrivals
+                        if (gk >= kBStages && !mbar_wait(&bars[kBEmpty + st], ((gk / kBStages) - 1) & 1, abort_s)) {
+                            ok = false;
+                            break;
+                        }
+                    } else if (kb < dkb) {
                         // U = u 2^10 for coordinates 64 kb .. 64 kb + 63, fp16 hi | lo; the inputs
                         // are fetched before waiting for the stage to free up
                         constexpr int NQ = F16 ? 8 : 16;
@@ -559,6 +609,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         uint32_t wp[BETA];
 #pragma unroll
                         for (int p = 0; p < BETA; ++p) wp[p] = 0u;
+                        uint32_t hp[RP ? 16 : 1], lp[RP ? 16 : 1];  // RP: fp16 hi | lo of 2^14 e, pairs
+                        float e_prev = 0.f;
 #pragma unroll
                         for (int l = 0; l < 32; ++l) {
                             const float y = __uint_as_float(a[l]) * yscale;
@@ -581,7 +633,24 @@ __global__ void __launch_bounds__(kBThreads, 1)
                                 }
                                 const float e = y - cv;
                                 ee = fmaf(e, e, ee);
+                                if constexpr (RP) {
+                                    if (l & 1) {
+                                        const float2 e2 = make_float2(e_prev * kEScale, e * kEScale);
+                                        const __half2 hh = __floats2half2_rn(e2.x, e2.y);
+                                        const float2 h2 = __half22float2(hh);
+                                        const __half2 ll = __floats2half2_rn(e2.x - h2.x, e2.y - h2.y);
+                                        hp[l >> 1] = *(const uint32_t *)&hh;
+                                        lp[l >> 1] = *(const uint32_t *)&ll;
+                                    } else {
+                                        e_prev = e;
+                                    }
+                                }
                             }
+                        }
+                        if constexpr (RP) {
+                            // in place: group g's 32 fp32 columns become its hi (16) and lo (16)
+                            tmem_st16(tl + 32 * g, hp);
+                            tmem_st16(tl + 32 * g + 16, lp);
                         }
                         if (valid) {
 #pragma unroll
@@ -614,25 +683,16 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     // d (a few 1e-5 of p at d = 1024), so projections with |p| < kSignRecheck are
                     // recomputed in double by the warp, from x, the codes, S and S'.
                     const int64_t vbase = v - lane;
-                    // exact path: 2^18 p = ACC_S 2^18 / ||ACC|| + ACC_c (columns 128 on)
-                    const float pscale = na > 0.f ? (float)(1 << (kUScaleLog2 + kRScaleLog2)) / na : 0.f;
+                    // a recheck reads the vector's codes from both column halves
+                    if (RP && !mbar_wait(&bars[kBCodes + (i & 1)], (i >> 1) & 1, abort_s)) {
+                        ok = false;
+                        break;
+                    }
 #pragma unroll 1
                     for (int g = gA; g < gB; ++g) {
                         uint32_t a[32];
                         tmem_ld32(tl + 32 * g, a);
                         tmem_ld_wait();
-                        if (exact) {
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                uint32_t b16[16];
-                                tmem_ld16(tl + 128 + 32 * g + 16 * hh, b16);
-                                tmem_ld_wait();
-#pragma unroll
-                                for (int l = 0; l < 16; ++l)
-                                    a[16 * hh + l] = __float_as_uint(
-                                        fmaf(__uint_as_float(a[16 * hh + l]), pscale, __uint_as_float(b16[l])));
-                            }
-                        }
                         uint32_t sw = 0, unc = 0;
 #pragma unroll
                         for (int l = 0; l < 32; ++l) {
@@ -657,6 +717,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         if (valid) signs[v * SWPT + g0 + g] = sw;
                     }
                 }
+                if (RP && c < G.nr) tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kBAccEmpty + slot]);
@@ -680,7 +741,7 @@ cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64
     const size_t smem = L.total + 1024;
     // the exact path for fp16 input with one rotation chunk; its code step split over eight warps
     // where it is heavy (keys; values of 3 or 4 bits)
-    const bool ex = F16 && G.nr == 1 && (!IS_KEY || (G.m <= 128 && G.m % 64 == 0));
+    const bool ex = F16 && G.nr == 1 && (!IS_KEY || G.ns == 1);
     const bool split = ex && (IS_KEY || BETA >= 3);
     auto kern = split ? compress_big_kernel<IS_KEY, BETA, F16, F16, F16>
                       : ex ? compress_big_kernel<IS_KEY, BETA, F16, F16, false>

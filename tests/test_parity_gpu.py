@@ -97,6 +97,18 @@ def test_compress_large_projection(tq):
     _compress_both(tq, x, R, S, 2, True)
 
 
+@pytest.mark.parametrize("m", [32, 96, 192, 256])
+def test_compress_wide_head_projection_widths(tq, m):
+    """d = 256 fp16 keys: one rotation chunk and one projection chunk of any width up to 256,
+    a ragged tail and several tiles per CTA."""
+    d = 256
+    R = synth.rotation(d, 31)
+    S = synth.gaussian(m, d, 32 + m)
+    x = synth.gaussian(128 * 148 + 300, d, 33).astype(np.float16)
+    for bits in (2, 3, 4):
+        _compress_both(tq, x, R, S, bits, True)
+
+
 # -------------------------------------------------------------------- scores
 
 def _oracle_cache(seed, d, m, bits, B, Hkv, T, f16=True):
