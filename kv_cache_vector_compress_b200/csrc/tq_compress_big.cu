@@ -91,42 +91,39 @@ struct BigGeom {
     __host__ __device__ int kb_per_tile() const { return nr * (d / 64) + ns * 2 * (d / 64); }
 };
 
-// Code of y against ascending boundaries b[0..2^BETA-2] (#{k : b[k] < y}) by a binary search
-// over register thresholds; t[p] receives bit p of the code.
+// The codebooks are symmetric (c[HL + k] = -c[HL - 1 - k], middle boundary 0, HL = 2^(BETA-1)),
+// so the code of y follows from its sign and the digits of m = #{k : e[k] < |y|} over the HL - 1
+// positive boundaries e[k] = b[HL + k]: the code is HL + m for y > 0 and HL - 1 - m otherwise, so
+// its top bit is [y > 0] and its bit j < BETA - 1 is m_j when y > 0, not m_j otherwise.
+// big_mag sets mb[j] = m_j by a binary search over thresholds held in registers.
 template <int BETA>
-__device__ __forceinline__ uint32_t big_bucket(float y, const float (&b)[16]) {
-    if constexpr (BETA == 1) {
-        return y > b[0] ? 1u : 0u;
-    } else if constexpr (BETA == 2) {
-        const uint32_t t1 = y > b[1];
-        const uint32_t t0 = y > (t1 ? b[2] : b[0]);
-        return (t1 << 1) | t0;
+__device__ __forceinline__ void big_mag(float u, const float *e, bool (&mb)[3]) {
+    if constexpr (BETA == 2) {
+        mb[0] = u > e[0];
     } else if constexpr (BETA == 3) {
-        const uint32_t t2 = y > b[3];
-        const uint32_t t1 = y > (t2 ? b[5] : b[1]);
-        const uint32_t t0 = y > (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0]));
-        return (t2 << 2) | (t1 << 1) | t0;
-    } else {
-        const uint32_t t3 = y > b[7];
-        const uint32_t t2 = y > (t3 ? b[11] : b[3]);
-        const uint32_t t1 = y > (t3 ? (t2 ? b[13] : b[9]) : (t2 ? b[5] : b[1]));
-        const uint32_t t0 = y > (t3 ? (t2 ? (t1 ? b[14] : b[12]) : (t1 ? b[10] : b[8]))
-                                    : (t2 ? (t1 ? b[6] : b[4]) : (t1 ? b[2] : b[0])));
-        return (t3 << 3) | (t2 << 2) | (t1 << 1) | t0;
+        mb[1] = u > e[1];
+        mb[0] = u > (mb[1] ? e[2] : e[0]);
+    } else if constexpr (BETA == 4) {
+        mb[2] = u > e[3];
+        mb[1] = u > (mb[2] ? e[5] : e[1]);
+        mb[0] = u > (mb[2] ? (mb[1] ? e[6] : e[4]) : (mb[1] ? e[2] : e[0]));
     }
 }
 
-// The same search with the boundaries read from shared memory (b_s[0..2^BETA-2]) by index, for
-// 3 and 4 bits, where the register form needs 3 and 11 selects per coordinate.
+// |c| = cm[m] from the digits of m (HL positive centroids in registers).
 template <int BETA>
-__device__ __forceinline__ uint32_t big_bucket_s(float y, const float *b_s) {
-    uint32_t idx = 0;
-#pragma unroll
-    for (int p = BETA - 1; p >= 0; --p) {
-        const uint32_t t = y > b_s[idx + (1u << p) - 1];
-        idx += t << p;
+__device__ __forceinline__ float big_cmag(const bool (&mb)[3], const float *cm) {
+    if constexpr (BETA == 1) {
+        return cm[0];
+    } else if constexpr (BETA == 2) {
+        return mb[0] ? cm[1] : cm[0];
+    } else if constexpr (BETA == 3) {
+        return mb[1] ? (mb[0] ? cm[3] : cm[2]) : (mb[0] ? cm[1] : cm[0]);
+    } else {
+        const float hi = mb[1] ? (mb[0] ? cm[7] : cm[6]) : (mb[0] ? cm[5] : cm[4]);
+        const float lo = mb[1] ? (mb[0] ? cm[3] : cm[2]) : (mb[0] ? cm[1] : cm[0]);
+        return mb[2] ? hi : lo;
     }
-    return idx;
 }
 
 __device__ __forceinline__ uint32_t hsplit2(float a, float b, bool lo) {
@@ -137,6 +134,10 @@ __device__ __forceinline__ uint32_t hsplit2(float a, float b, bool lo) {
 }
 
 constexpr float kSignRecheck = 1e-4f;  // |p| below which a sign is recomputed exactly
+// The residual form has no cancelling O(1) terms: its error is the fp32 rounding of y carried
+// through S' plus that of the d-term sum of S'_a e (a few 1e-6 at d <= 256 even with truncating
+// accumulation), so it rechecks only below 2e-5.
+constexpr float kSignRecheckResidual = 2e-5f;
 constexpr float kPUnscaleInv = (float)(1 << (kUScaleLog2 + kRScaleLog2));  // ACC = p 2^18
 constexpr float kEScale = (float)(1 << kCorrScaleLog2);  // residual operand 2^14 e
 
@@ -542,19 +543,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const int r = 32 * q4 + lane;
         const int hf = SPLIT ? (warp - kEpi0) >> 2 : 0;  // column half of this warp
         constexpr int NHF = SPLIT ? 2 : 1;
-        float bnd_r[16], cen_r[16];
+        constexpr int HL = 1 << (BETA - 1);
+        float edge[HL > 1 ? HL - 1 : 1], cmag[HL];  // positive boundaries; 2^14 |c| (keys)
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            bnd_r[k] = bnd_s[k];
-            cen_r[k] = cen_s[k];
-        }
+        for (int k = 0; k < HL - 1; ++k) edge[k] = bnd_s[HL + k];
+#pragma unroll
+        for (int k = 0; k < HL; ++k) cmag[k] = cen_s[HL + k] * kEScale;
         constexpr float kYUnscale = 1.0f / (float)(1 << (kUScaleLog2 + kRScaleLog2));
         int gc = 0;
         bool ok = true;
         for (int i = 0; ok && i < my_tiles; ++i) {
             const int64_t v = (blockIdx.x + (int64_t)i * gridDim.x) * kBRows + r;
             const bool valid = v < n;
-            float ee = 0.f;
+            float2 ee2 = make_float2(0.f, 0.f);  // (2^14 ||y - c||)^2 over even | odd coordinates
             float na = 0.f;  // exact path: ||ACC|| of the rotation chunk (2^8 ||x||)
             for (int c = 0; c < NC; ++c, ++gc) {
                 const int slot = gc & 1;
@@ -600,53 +601,60 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     if (valid && hf == 0) norm[v] = f32_to_f16_bits(na * (1.0f / (float)(1 << kRScaleLog2)));
                 }
                 if (c < G.nr) {
-                    // codes of rotated coordinates 32 (g0 + g) .. + 31, planar words
+                    // codes of rotated coordinates 32 (g0 + g) .. + 31, planar words.  y = ACC yscale
+                    // is compared as ACC against the boundaries scaled by 1 / yscale; a zero vector
+                    // compares its zero accumulator against the unscaled ones (y = 0).
+                    const float sc = yscale > 0.f ? (exact ? na : 1.0f / kYUnscale) : 1.f;
+                    float ep[HL > 1 ? HL - 1 : 1];
+#pragma unroll
+                    for (int k = 0; k < HL - 1; ++k) ep[k] = edge[k] * sc;
+                    const float ys14 = yscale * kEScale;  // ACC -> 2^14 y
 #pragma unroll 1
                     for (int g = gA; g < gB; ++g) {
                         uint32_t a[32];
                         tmem_ld32(tl + 32 * g, a);
                         tmem_ld_wait();
-                        uint32_t wp[BETA];
+                        // words of [y > 0] and of the magnitude digits; the code planes follow per word
+                        uint32_t sgn = 0u, mbw[BETA > 1 ? BETA - 1 : 1];
 #pragma unroll
-                        for (int p = 0; p < BETA; ++p) wp[p] = 0u;
+                        for (int j = 0; j < BETA - 1; ++j) mbw[j] = 0u;
                         uint32_t hp[RP ? 16 : 1], lp[RP ? 16 : 1];  // RP: fp16 hi | lo of 2^14 e, pairs
-                        float e_prev = 0.f;
 #pragma unroll
-                        for (int l = 0; l < 32; ++l) {
-                            const float y = __uint_as_float(a[l]) * yscale;
-                            // shared-memory tables on the split exact path; elsewhere shared memory
-                            // is busy with both MMA operands, and the register selects are faster
-                            const uint32_t idx =
-                                (SPLIT && BETA >= 3) ? big_bucket_s<BETA>(y, bnd_s) : big_bucket<BETA>(y, bnd_r);
+                        for (int k = 0; k < 16; ++k) {
+                            float es[2];
 #pragma unroll
-                            for (int p = 0; p < BETA; ++p) wp[p] |= ((idx >> p) & 1u) << l;
-                            if (IS_KEY) {
-                                // split exact path, 3 MSE bits: one shared-memory read (the 8
-                                // centroids in 8 banks) instead of a chain of 7 selects
-                                float cv;
-                                if constexpr (SPLIT && BETA >= 3) {
-                                    cv = cen_s[idx];
-                                } else {
-                                    cv = cen_r[0];
+                            for (int u = 0; u < 2; ++u) {
+                                const int l = 2 * k + u;
+                                const float av = __uint_as_float(a[l]), ua = fabsf(av);
+                                const bool pos = av > 0.f;
+                                bool mb[3] = {false, false, false};
+                                big_mag<BETA>(ua, ep, mb);
+                                if (pos) sgn |= 1u << l;
 #pragma unroll
-                                    for (int k = 1; k < (1 << BETA); ++k) cv = idx == (uint32_t)k ? cen_r[k] : cv;
+                                for (int j = 0; j < BETA - 1; ++j)
+                                    if (mb[j]) mbw[j] |= 1u << l;
+                                if (IS_KEY) {
+                                    // y - c = sign(y) (|y| - |c|), 2^14 scaled
+                                    const float em = fmaf(ua, ys14, -big_cmag<BETA>(mb, cmag));
+                                    es[u] = pos ? em : -em;
                                 }
-                                const float e = y - cv;
-                                ee = fmaf(e, e, ee);
+                            }
+                            if (IS_KEY) {
+                                const float2 e2 = make_float2(es[0], es[1]);
+                                ee2 = __ffma2_rn(e2, e2, ee2);
                                 if constexpr (RP) {
-                                    if (l & 1) {
-                                        const float2 e2 = make_float2(e_prev * kEScale, e * kEScale);
-                                        const __half2 hh = __floats2half2_rn(e2.x, e2.y);
-                                        const float2 h2 = __half22float2(hh);
-                                        const __half2 ll = __floats2half2_rn(e2.x - h2.x, e2.y - h2.y);
-                                        hp[l >> 1] = *(const uint32_t *)&hh;
-                                        lp[l >> 1] = *(const uint32_t *)&ll;
-                                    } else {
-                                        e_prev = e;
-                                    }
+                                    const __half2 hh = __floats2half2_rn(e2.x, e2.y);
+                                    const float2 h2 = __half22float2(hh);
+                                    const __half2 ll = __floats2half2_rn(e2.x - h2.x, e2.y - h2.y);
+                                    hp[k] = *(const uint32_t *)&hh;
+                                    lp[k] = *(const uint32_t *)&ll;
                                 }
                             }
                         }
+                        uint32_t wp[BETA];
+                        wp[BETA - 1] = sgn;
+#pragma unroll
+                        for (int j = 0; j < BETA - 1; ++j) wp[j] = ~(mbw[j] ^ sgn);
                         if constexpr (RP) {
                             // in place: group g's 32 fp32 columns become its hi (16) and lo (16)
                             tmem_st16(tl + 32 * g, hp);
@@ -660,6 +668,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     if (IS_KEY && c == G.nr - 1) {
                         // every code word of this tile is out: release the correction operands.
                         // Exact path: half 1 hands its part of ||y - c||^2 to half 0 first.
+                        float ee = (ee2.x + ee2.y) * (1.0f / (kEScale * kEScale));
                         if (SPLIT && hf == 1) {
                             xe_s[(i & 1) * kBRows + r] = ee;
                             __syncwarp();
@@ -679,9 +688,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     }
                 } else {
                     // signs of the projections 32 (g0 + g) .. + 31: sign(S u - S' c) = sign(ACC).
-                    // The two terms are O(1) and cancel to p; the accumulator's rounding grows with
-                    // d (a few 1e-5 of p at d = 1024), so projections with |p| < kSignRecheck are
-                    // recomputed in double by the warp, from x, the codes, S and S'.
+                    // In the two-term form the terms are O(1) and cancel to p; the accumulator's
+                    // rounding grows with d (a few 1e-5 of p at d = 1024), so projections with
+                    // |p| < kSignRecheck (kSignRecheckResidual in the residual form) are recomputed
+                    // in double by the warp, from x, the codes, S and S'.
                     const int64_t vbase = v - lane;
                     // a recheck reads the vector's codes from both column halves
                     if (RP && !mbar_wait(&bars[kBCodes + (i & 1)], (i >> 1) & 1, abort_s)) {
@@ -698,7 +708,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         for (int l = 0; l < 32; ++l) {
                             const float pv = __uint_as_float(a[l]);
                             sw |= (uint32_t)(pv >= 0.f) << l;
-                            unc |= (uint32_t)(fabsf(pv) < kSignRecheck * kPUnscaleInv) << l;
+                            unc |= (uint32_t)(fabsf(pv) < (RP ? kSignRecheckResidual : kSignRecheck) * kPUnscaleInv) << l;
                         }
                         if (!valid) unc = 0;
                         uint32_t pend = __ballot_sync(kFull, unc != 0);
@@ -743,9 +753,11 @@ cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64
     // where it is heavy (keys; values of 3 or 4 bits)
     const bool ex = F16 && G.nr == 1 && (!IS_KEY || G.ns == 1);
     const bool split = ex && (IS_KEY || BETA >= 3);
-    auto kern = split ? compress_big_kernel<IS_KEY, BETA, F16, F16, F16>
-                      : ex ? compress_big_kernel<IS_KEY, BETA, F16, F16, false>
-                           : compress_big_kernel<IS_KEY, BETA, F16, false, false>;
+    auto kern = compress_big_kernel<IS_KEY, BETA, F16, false, false>;
+    if (split) kern = compress_big_kernel<IS_KEY, BETA, F16, F16, F16>;
+    if constexpr (!IS_KEY) {
+        if (ex && !split) kern = compress_big_kernel<IS_KEY, BETA, F16, F16, false>;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
