@@ -26,6 +26,10 @@
 // (S u = S R^T y), so the epilogue writes 2^14 e = 2^14 (y - c[idx]) as fp16 hi | lo back into
 // the rotation slot and the projection chunk multiplies that TMEM operand by (S' 2^4)(hi + lo),
 // three products per k-step into one accumulator; the converters build no correction blocks.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
 #include "tq_common.cuh"
 #include "tq_internal.cuh"
 #include "tq_sm100.cuh"
@@ -190,7 +194,8 @@ __device__ __noinline__ double exact_projection(const Prepared &P, const BigGeom
 
 template <bool IS_KEY, int BETA, bool F16, bool EX, bool SPLIT>
 __global__ void __launch_bounds__(kBThreads, 1)
-    compress_big_kernel(Prepared P, BigGeom G, const void *__restrict__ xin, int64_t n, uint32_t *__restrict__ codes,
+    compress_big_kernel(const __grid_constant__ CUtensorMap xmap, Prepared P, BigGeom G, const void *__restrict__ xin,
+                        int64_t n, uint32_t *__restrict__ codes,
                         uint32_t *__restrict__ signs, uint16_t *__restrict__ norm, uint16_t *__restrict__ rnorm,
                         int32_t *__restrict__ dev_status) {
     const BigSmem L = big_smem_layout();
@@ -226,7 +231,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kBStages; ++s) {
-            mbar_init(&bars[kBFull + s], 5);  // the four converter warps of a group + the B copy
+            // the four converter warps of a group + the B copy; exact path: the copies of A and B
+            mbar_init(&bars[kBFull + s], EX ? 1 : 5);
             mbar_init(&bars[kBEmpty + s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -271,6 +277,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
             const size_t slo = (size_t)G.m * d * 2;
             int gk = 0, issued = 0;
             bool ok = true;
+            if (EX) prefetch_tmap(&xmap);
             for (int i = 0; ok && i < my_tiles; ++i)
                 for (int c = 0; ok && c < NC; ++c) {
                     const int w = G.width(c), n0 = G.n0(c), nkb = nkb_of(c);
@@ -294,7 +301,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
                             lo = slo;
                         }
                         uint8_t *dst = sm + L.stage + st * kBStage + 2 * kATile;
-                        mbar_arrive_expect_tx(&bars[kBFull + st], 2 * bytes);
+                        // exact path: A is the fp16 input tile itself, 128 rows x 64 coordinates in
+                        // the 128-byte swizzle (rows past n read as zeros)
+                        const bool xa = EX && c < G.nr;
+                        mbar_arrive_expect_tx(&bars[kBFull + st], 2 * bytes + (xa ? kATile : 0u));
+                        if (xa)
+                            tma_load_2d(sm + L.stage + st * kBStage, &xmap, &bars[kBFull + st], 64 * kb,
+                                        (int)((blockIdx.x + (int64_t)i * gridDim.x) * kBRows));
                         bulk_load(dst, src, bytes, &bars[kBFull + st]);
                         bulk_load(dst + kBTileMax, src + lo, bytes, &bars[kBFull + st]);
                         issued = gk + 1;
@@ -384,6 +397,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
     } else if (warp < kEpi0) {
         // -------------------------------------------------------- A tiles, one vector per thread
+        // (the exact path's producer loads A by TMA: no converter work)
+        if constexpr (!EX) {
         const int cg = SPLIT ? 0 : (warp - kCvtWarp0) >> 2;  // group: K-block steps gk with gk % 2 == cg
         const int r = (threadIdx.x - kCvtWarp0 * 32) & 127;  // the vector this thread converts
         const uint32_t rowb = (uint32_t)r * 128;
@@ -536,6 +551,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     if (lane == 0) mbar_arrive(&bars[kBFull + st]);
                 }
             }
+        }
         }
     } else {
         // -------------------------------------------------------- epilogue, one vector per thread
@@ -744,6 +760,18 @@ __global__ void __launch_bounds__(kBThreads, 1)
     if (threadIdx.x == 0 && *abort_s && dev_status) atomicExch(dev_status, (int)TQ_ERR_TIMEOUT);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 big_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }
+    return fn;
+}
+
 template <bool IS_KEY, int BETA, bool F16>
 cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64_t n, uint32_t *codes, uint32_t *signs,
                        uint16_t *norm, uint16_t *rnorm, int32_t *dev_status, cudaStream_t s) {
@@ -751,12 +779,27 @@ cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64
     const size_t smem = L.total + 1024;
     // the exact path for fp16 input with one rotation chunk; its code step split over eight warps
     // where it is heavy (keys; values of 3 or 4 bits)
-    const bool ex = F16 && G.nr == 1 && (!IS_KEY || G.ns == 1);
+    const bool ex = F16 && G.nr == 1 && (!IS_KEY || G.ns == 1) && n <= (int64_t)INT32_MAX;
     const bool split = ex && (IS_KEY || BETA >= 3);
     auto kern = compress_big_kernel<IS_KEY, BETA, F16, false, false>;
     if (split) kern = compress_big_kernel<IS_KEY, BETA, F16, F16, F16>;
     if constexpr (!IS_KEY) {
         if (ex && !split) kern = compress_big_kernel<IS_KEY, BETA, F16, F16, false>;
+    }
+    // exact path: a tensor map over the fp16 rows (n x d), 64 x 128 boxes in the 128-byte swizzle
+    CUtensorMap xmap;
+    memset(&xmap, 0, sizeof(xmap));
+    if (ex) {
+        auto encode = big_encode_fn();
+        if (!encode) return cudaErrorNotSupported;
+        cuuint64_t dims[2] = {(cuuint64_t)G.d, (cuuint64_t)n};
+        cuuint64_t strides[1] = {(cuuint64_t)G.d * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)kBRows};
+        cuuint32_t estr[2] = {1, 1};
+        if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -765,7 +808,7 @@ cudaError_t launch_big(const Prepared &P, const BigGeom &G, const void *x, int64
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t ntiles = (n + kBRows - 1) / kBRows;
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    kern<<<grid, kBThreads, smem, s>>>(P, G, x, n, codes, signs, norm, rnorm, dev_status);
+    kern<<<grid, kBThreads, smem, s>>>(xmap, P, G, x, n, codes, signs, norm, rnorm, dev_status);
     return cudaGetLastError();
 }
 
