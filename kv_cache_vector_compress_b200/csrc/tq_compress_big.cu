@@ -19,13 +19,14 @@
 // tiles (two groups taking alternate K-blocks), 10..13 run the epilogue.  Two TMEM slots of
 // 256 columns keep one chunk's epilogue under the next chunk's MMAs.
 // fp16 input with d <= 256 (one rotation chunk; keys also m <= 256) takes the input itself as the
-// A operand: fp16 is exact, so x (R 2^8)(hi + lo) needs two products per k-step, the converters
-// only copy the rows into the swizzled stage, and the epilogue takes ||x|| = ||ACC|| / 2^8 from
-// the rotation accumulator (R orthogonal, to the 2^-22 of its split) before coding
-// y = ACC / ||ACC||.  Keys then project the residual: p = S u - S' c[idx] = S' (y - c[idx])
-// (S u = S R^T y), so the epilogue writes 2^14 e = 2^14 (y - c[idx]) as fp16 hi | lo back into
-// the rotation slot and the projection chunk multiplies that TMEM operand by (S' 2^4)(hi + lo),
-// three products per k-step into one accumulator; the converters build no correction blocks.
+// A operand: fp16 is exact, so x (R 2^8)(hi + lo) needs two products per k-step, warp 0 loads the
+// rows by TMA into the swizzled stage beside the B tiles (the converter warps have no work), and
+// the epilogue takes ||x|| = ||ACC|| / 2^8 from the rotation accumulator (R orthogonal, to the
+// 2^-22 of its split) before coding y = ACC / ||ACC||.  Keys then project the residual:
+// p = S u - S' c[idx] = S' (y - c[idx]) (S u = S R^T y), so the epilogue writes
+// 2^14 e = 2^14 (y - c[idx]) as fp16 hi | lo back into the rotation slot and the projection chunk
+// multiplies that TMEM operand by (S' 2^4)(hi + lo), three products per k-step into one
+// accumulator; there are no correction blocks.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -213,9 +214,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int KWPT = BETA * (d / 32);
     const int SWPT = G.m / 32;
     const int NC = G.nchunks();
-    // EX: A = the fp16 input itself (see the header).  SPLIT (exact path with a heavier code step):
-    // one converter group (warps 2..5) takes every K-block and eight epilogue warps (6..13, two
-    // column halves) code each tile.
+    // EX: A = the fp16 input itself, loaded by TMA (see the header); warps 2 .. kEpi0 - 1 idle.
+    // SPLIT (exact path with a heavier code step): eight epilogue warps (6..13, two column halves)
+    // code each tile.
     constexpr bool exact = EX;
     // RP (exact keys): the projection is p = S' e of the residual e = y - c[idx], which the
     // epilogue writes back into the rotation slot (fp16 hi | lo of 2^14 e) as the A operand of the
